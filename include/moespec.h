@@ -1,0 +1,207 @@
+/*
+ * moespec -- MoE verify layer and greedy speculative verification for
+ * NVIDIA B200 (sm_100a).  C ABI of libmoespec.so.
+ *
+ * The operation these calls implement is the hot path of the jina-ocr-v1
+ * document parser's decoder as its pages describe it:
+ *  - a mixture-of-experts decoder layer with 64 routed experts, two shared
+ *    experts and top-6 routing (clawpit.io, "Lean architecture with a
+ *    compressed encoder"; aikraft.ru, "Архитектура и эффективность"),
+ *  - run over the K+1 positions that FastMTP speculative decoding verifies
+ *    (K = 3 drafts), followed by greedy verification: accept the longest
+ *    prefix of drafts that matches the verifier's own picks and commit one
+ *    more token of the verifier's (jina.ai, "Modèle et entraînement";
+ *    clawpit.io, "Speculative decoding without accuracy loss").
+ * The pages define no programming interface; the calls below follow the
+ * steps of that statement.
+ *
+ * Conventions for every call
+ *  - Pointers: every tensor argument is a DEVICE pointer unless stated, in
+ *    row-major layout, and must be 16-byte aligned.  bf16 tensors hold IEEE
+ *    bfloat16 bit patterns.  The caller owns every buffer; the library never
+ *    allocates, frees or retains device memory during a call.
+ *  - Scratch: calls that need scratch take (ws, ws_bytes), sized by the
+ *    matching *_workspace_size() query; contents need no initialisation and
+ *    are clobbered.  ws must not be shared by calls that may overlap.
+ *  - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).
+ *    Every call is asynchronous on that stream and never synchronises the
+ *    host.  Kernels are launched with programmatic dependent launch, so a
+ *    call may begin while the previous kernel on the stream drains; each
+ *    kernel waits for its predecessor before touching memory.
+ *  - Errors: arguments are validated on the host before anything is
+ *    launched; a bad argument returns MS_ERR_INVALID_ARG / MS_ERR_UNSUPPORTED
+ *    / MS_ERR_WORKSPACE and launches nothing.  A failed launch returns
+ *    MS_ERR_CUDA (details via ms_last_cuda_error_string).  Device-side
+ *    conditions (a bounded wait that ran out, an out-of-range index seen by
+ *    a kernel) are recorded in a status word inside the caller's workspace
+ *    and read with ms_device_status(); the kernel then skips the affected
+ *    work instead of trapping.
+ *  - Sizes: 1 <= k <= E <= 256; H % 128 == 0; I % 128 == 0; 1 <= K <= 8.
+ */
+#ifndef MOESPEC_H
+#define MOESPEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MS_API __attribute__((visibility("default")))
+#else
+#define MS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MS_OK = 0,
+    MS_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, bad enum    */
+    MS_ERR_UNSUPPORTED = -2,   /* valid but outside the supported shape set   */
+    MS_ERR_WORKSPACE = -3,     /* ws missing or smaller than the size query   */
+    MS_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed            */
+    MS_ERR_TIMEOUT = -5,       /* a device-side bounded wait ran out           */
+    MS_ERR_DEVICE_INDEX = -6   /* a kernel saw an index outside its range      */
+} ms_status;
+
+typedef enum { MS_F32 = 0, MS_BF16 = 1 } ms_dtype;
+
+/* ---------------------------------------------------------------------- */
+/* a0  RMSNorm of the residual stream (the layer's normalised input).
+ * xhat_bf16[t,h] = bf16( a[t,h] / sqrt(mean_h(a[t,:]^2) + eps) * gamma[h] )
+ * a: [T,H] fp32.  gamma: [H] fp32 or NULL (= 1).  xhat_bf16: [T,H] bf16.
+ * The pages do not describe the normalisation; it is the conventional
+ * pre-MoE RMSNorm of a DeepSeek-style decoder block. */
+MS_API ms_status moe_rmsnorm(const float* a, const float* gamma, int T, int H, float eps,
+                      void* xhat_bf16, void* stream);
+
+/* a1  Router: fp32 softmax over E experts and top-k selection
+ * (top-6 of 64 routed experts: clawpit.io, "Lean architecture ...").
+ * z[t,e] = sum_h xhat[t,h] * w_router[e,h] (+ logit_bias[t,e]), fp32.
+ * topk_idx[t,0..k-1]: the k largest z in descending order, equal values
+ *   broken towards the lower expert index.
+ * topk_w[t,j] = softmax(z[t,:])[topk_idx[t,j]], divided by the sum of the
+ *   k selected probabilities when renormalize != 0.
+ * xhat: [T,H] bf16.  w_router: [E,H] fp32.  logit_bias: [T,E] fp32 or NULL.
+ * topk_idx: [T,k] int32.  topk_w: [T,k] fp32.  No scratch. */
+MS_API ms_status moe_route_topk(const void* xhat, const float* w_router, const float* logit_bias,
+                         int T, int H, int E, int k, int renormalize,
+                         int32_t* topk_idx, float* topk_w, void* stream);
+
+/* a2  Permutation: group the T*k (token, slot) pairs by expert, ordered by
+ * (expert, token) -- a stable counting sort, bit-exact and deterministic.
+ * expert_offsets: [E+1] int32, expert e owns rows [off[e], off[e+1]).
+ * perm_token: [T*k] int32, token of each grouped row.
+ * slot_of: [T,k] int32, grouped row of pair (t,j).
+ * Scratch: moe_permute_workspace_size(T,k,E) bytes (0 is returned, and ws
+ * may be NULL, when T*k <= 4096).  Out-of-range expert ids are skipped and
+ * flagged (MS_ERR_DEVICE_INDEX) when ws is given. */
+MS_API size_t moe_permute_workspace_size(int T, int k, int E);
+MS_API ms_status moe_permute(const int32_t* topk_idx, int T, int k, int E,
+                      int32_t* expert_offsets, int32_t* perm_token, int32_t* slot_of,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* a3  Expert FFN: every routed row and the shared experts, SwiGLU.
+ * For grouped row r of expert e (token t = perm_token[r]):
+ *   g = W_g[e] x_t, u = W_u[e] x_t, h = silu(g) * u (rounded to bf16),
+ *   y_perm[r,:] = W_d[e] h            (fp32 accumulation throughout)
+ * y_shared[t,:] = sum_s W_d^s (silu(W_g^s x_t) * (W_u^s x_t)).
+ * xhat: [T,H] bf16.  w_gate_up: [E,2I,H] bf16 (rows 0..I-1 gate, I..2I-1
+ * up).  w_down: [E,H,I] bf16.  ws_gate_up: [S,2I,H] bf16, ws_down: [S,H,I]
+ * bf16 (both NULL iff S == 0).  y_perm: [T*k,H] of y_perm_dtype.
+ * y_shared: [T,H] fp32 (may be NULL iff S == 0).
+ * Tensor-core grouped GEMMs (tcgen05 + TMEM, TMA-fed).  T <= 128 uses a
+ * weight-streaming schedule balanced over all SMs; larger T a tiled one.
+ * Scratch: moe_expert_ffn_workspace_size(...) bytes; the status word of
+ * the bounded waits lives at its start (see ms_device_status). */
+MS_API size_t moe_expert_ffn_workspace_size(int T, int H, int E, int I, int S, int k);
+MS_API ms_status moe_expert_ffn(const void* xhat, const int32_t* expert_offsets, const int32_t* perm_token,
+                         const void* w_gate_up, const void* w_down,
+                         const void* ws_gate_up, const void* ws_down,
+                         int T, int H, int E, int I, int S, int k,
+                         void* y_perm, ms_dtype y_perm_dtype, float* y_shared,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* a4  Combine: gate-weighted un-permute plus residual.
+ * out[t,:] = sum_{j<k} topk_w[t,j] * y_perm[slot_of[t,j],:] + y_shared[t,:]
+ *            + residual[t,:]            (fp32, in that order)
+ * y_perm: [T*k,H] fp32 or bf16.  y_shared, residual: [T,H] fp32 or NULL.
+ * out: [T,H] fp32.  out_bf16: [T,H] bf16 copy or NULL.  No scratch. */
+MS_API ms_status moe_combine(const void* y_perm, ms_dtype y_perm_dtype, const float* y_shared,
+                      const int32_t* slot_of, const float* topk_w, const float* residual,
+                      int T, int H, int k, float* out, void* out_bf16, void* stream);
+
+/* a5  Vocab head for the verify rows: logits[t,v] = sum_h xhat[t,h] w_lm[v,h].
+ * xhat: [T,H] bf16, w_lm: [V,H] bf16, logits: [T,V] bf16 (fp32 accumulate).
+ * V % 128 == 0.  Tensor-core GEMM; T is processed 128 rows at a time.
+ * Scratch: lm_head_workspace_size(T,H,V) bytes. */
+MS_API size_t lm_head_workspace_size(int T, int H, int V);
+MS_API ms_status lm_head_logits(const void* xhat, const void* w_lm, int T, int H, int V,
+                         void* logits_bf16, void* ws, size_t ws_bytes, void* stream);
+
+/* a6  Greedy verification of one speculative step for B sequences
+ * (jina.ai, "Modèle et entraînement"; clawpit.io, "Speculative decoding
+ * without accuracy loss"; tau counts the bonus token: jina.ai, "Décodage
+ * spéculatif sur un L4").
+ * logits: [B,K+1,V] of logits_dtype; row j scores the token after position j
+ *   (position 0 = last committed token, 1..K = the drafts).
+ * draft: [B,K] int32.
+ * argmax[b,j] = argmax_v logits[b,j,v], lowest index among equal maxima;
+ * n = longest m <= K with draft[b,i] == argmax[b,i] for all i < m;
+ * committed[b,:] = draft[b,0..n-1], argmax[b,n], then -1 padding;
+ * n_committed[b] = n + 1, always in 1..K+1.
+ * argmax, committed: [B,K+1] int32.  n_committed: [B] int32.
+ * Scratch: spec_verify_workspace_size(B,K,V) bytes (partial maxima). */
+MS_API size_t spec_verify_workspace_size(int B, int K, int V);
+MS_API ms_status spec_verify_greedy(const void* logits, ms_dtype logits_dtype, const int32_t* draft,
+                             int B, int K, int V, int32_t* argmax, int32_t* committed,
+                             int32_t* n_committed, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Whole layer in hot-path order: rmsnorm -> route -> permute -> expert FFN
+ * -> combine.  a: [T,H] fp32 residual input, out: [T,H] fp32.  The
+ * intermediates live in ws (moe_layer_workspace_size bytes). */
+MS_API size_t moe_layer_workspace_size(int T, int H, int E, int I, int S, int k);
+MS_API ms_status moe_layer_forward(const float* a, const float* w_router, const float* logit_bias,
+                            const void* w_gate_up, const void* w_down,
+                            const void* ws_gate_up, const void* ws_down,
+                            int T, int H, int E, int I, int S, int k, int renormalize,
+                            float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Device status word kept at the start of a workspace given to
+ * moe_expert_ffn, lm_head_logits or moe_layer_forward.  Each of those calls
+ * clears it (stream-ordered) before its first kernel, so it holds the first
+ * device-side condition of the most recent call on that workspace.  This
+ * synchronises `stream`, returns the word (MS_OK if nothing was recorded)
+ * and clears it. */
+MS_API ms_status ms_device_status(void* ws, void* stream);
+
+/* Bounded-wait limit used by every device-side spin (default 1e9 ns). */
+MS_API void ms_set_wait_limit_ns(uint64_t ns);
+MS_API uint64_t ms_get_wait_limit_ns(void);
+
+/* Self-test of the bounded wait: one kernel spins until *flag == expect or
+ * the wait limit passes, then writes MS_OK or MS_ERR_TIMEOUT to *status
+ * (device int32).  flag, status: device pointers. */
+MS_API ms_status ms_debug_bounded_wait(const int32_t* flag, int32_t expect, int32_t* status,
+                                void* stream);
+
+/* Launch tracing: when enabled, every kernel this library launches is
+ * bracketed by a pair of CUDA events (recorded on the launching stream, so
+ * they also work inside stream capture).  ms_trace_read returns, after the
+ * stream has completed, the kernel name and duration of entry i. */
+MS_API ms_status ms_trace_enable(int capacity);
+MS_API void ms_trace_disable(void);
+MS_API void ms_trace_reset(void);
+MS_API int ms_trace_count(void);
+MS_API ms_status ms_trace_read(int i, const char** kernel_name, float* ms);
+
+MS_API const char* ms_status_string(ms_status s);
+MS_API const char* ms_last_cuda_error_string(void);
+MS_API int ms_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOESPEC_H */

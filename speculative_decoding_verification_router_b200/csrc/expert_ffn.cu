@@ -1,0 +1,977 @@
+// a3 (and a5): grouped SwiGLU expert GEMMs on the 5th-generation tensor cores.
+//
+// One persistent, warp-specialised kernel template serves every contraction
+// of the layer: GEMM1 (gate/up projections + SwiGLU), GEMM2 (down
+// projection) and the vocab head.  Warp 0 issues TMA loads (128-byte
+// swizzled tiles, no multicast), warp 1 issues tcgen05.mma from one thread
+// into TMEM accumulators (two buffers, so the epilogue of one tile overlaps
+// the main loop of the next), warps 2..5 drain TMEM with tcgen05.ld.
+//
+// Two schedules:
+//  * streaming (verify-sized T <= 128): the weights are the M = 128 operand
+//    and the tokens of one expert the N operand (N = rows rounded up to 16).
+//    The work -- every (group, 128-feature tile, 64-wide k-step) -- is
+//    divided into equal contiguous ranges of k-steps, one per CTA, so every
+//    SM streams the same number of weight bytes ("stream-K").  A tile split
+//    between CTAs is finished by the last CTA to arrive, which sums the fp32
+//    partials in CTA order (deterministic, no waiting on other CTAs).
+//    For GEMM1 the gate and up rows of the same 128 features accumulate into
+//    two TMEM buffers in the same lanes, so SwiGLU is done in registers.
+//  * tiled (prefill-sized T): the tokens of one expert are the M = 128
+//    operand and the weights the N operand; for GEMM1 the N = 256 tile is
+//    128 gate rows followed by the matching 128 up rows, so each thread holds
+//    both halves of its token row and applies SwiGLU in registers.
+// Shared experts form one extra group whose intermediate width is S*I: two
+// SwiGLU experts equal one expert with the intermediates concatenated.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "ms_sm100.cuh"
+
+namespace ms {
+
+using namespace sm100;
+
+constexpr int BM = 128;                  // MMA M
+constexpr int BK = 64;                   // k per stage = one 128-byte swizzle row
+constexpr int TILE_BYTES = BM * BK * 2;  // 16 KB: 128 rows x 64 bf16
+constexpr int TOKBOX = 16;               // token rows per TMA box (streaming)
+constexpr int NTHREADS = 192;
+constexpr int MAX_GROUPS = 257;
+constexpr int TMEM_COLS = 512;
+constexpr int SMEM_BUDGET = 210 * 1024;
+
+enum Mode : int { G1_STREAM = 0, G2_STREAM = 1, LM_STREAM = 2, G1_TILED = 3, G2_TILED = 4 };
+
+struct Maps {
+    CUtensorMap w_a;     // routed weights  [E][rows][K] (or [1][V][H] for the vocab head)
+    CUtensorMap w_s;     // shared weights  [S][rows][K]
+    CUtensorMap tok_r;   // routed token operand [rows][K]
+    CUtensorMap tok_s;   // shared token operand [rows][K]
+};
+
+struct Params {
+    int T, H, E, I, S, k, V;
+    int bn;                        // tiled GEMM2 output tile width (256 or 128)
+    const int32_t* offsets;        // [E+1]; nullptr for the vocab head
+    __nv_bfloat16* h_perm;         // [rows][I]
+    __nv_bfloat16* h_sh;           // [T][S*I]
+    void* y_perm;                  // [T*k][H] fp32 or bf16
+    int y_bf16;
+    float* y_sh;                   // [T][H]
+    __nv_bfloat16* logits;         // [T][V]
+    float* partials;               // 2 slots per CTA (streaming)
+    int32_t* counters;             // one per tile (streaming)
+    int32_t* status;
+    int max_tiles;                 // tiles per group upper bound (counter stride)
+    uint64_t wait_limit_ns;
+};
+
+template <int MODE>
+struct Cfg {
+    static constexpr bool kStream = MODE <= LM_STREAM;
+    static constexpr bool kG1 = MODE == G1_STREAM || MODE == G1_TILED;
+};
+
+template <int MODE, int NMAX>
+struct Layout {
+    static constexpr int A_BYTES = Cfg<MODE>::kStream ? (Cfg<MODE>::kG1 ? 2 : 1) * TILE_BYTES : TILE_BYTES;
+    static constexpr int B_BYTES = Cfg<MODE>::kStream ? NMAX * BK * 2 : 2 * TILE_BYTES;
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE;
+    static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+    static constexpr int SMEM = STAGES * STAGE + 1024;
+    static_assert(STAGE % 1024 == 0, "stage buffers must stay 1024-byte aligned");
+    static_assert(STAGES >= 2, "pipeline needs two stages");
+};
+
+// ------------------------------------------------------------ schedule
+struct Sched {
+    int ngroups;
+    int prefix[MAX_GROUPS + 1];   // units before group g
+    int rows[MAX_GROUPS];
+    int row0[MAX_GROUPS];
+};
+
+template <int MODE>
+__device__ __forceinline__ int group_ktiles(const Params& p, int g) {
+    const bool shared = p.offsets != nullptr && g == p.E;
+    if (MODE == G1_STREAM || MODE == G1_TILED || MODE == LM_STREAM) return p.H / BK;
+    return (shared ? p.S * p.I : p.I) / BK;   // GEMM2: K = intermediate width
+}
+
+template <int MODE>
+__device__ __forceinline__ int group_ntiles(const Params& p, int g) {
+    const bool shared = p.offsets != nullptr && g == p.E;
+    if (MODE == LM_STREAM) return p.V / BM;
+    if (MODE == G1_STREAM || MODE == G1_TILED) return (shared ? p.S * p.I : p.I) / BM;
+    if (MODE == G2_STREAM) return p.H / BM;
+    return p.H / p.bn;   // G2_TILED
+}
+
+template <int MODE>
+__device__ void build_schedule(const Params& p, Sched& s) {
+    const int tid = threadIdx.x;
+    if (p.offsets == nullptr) {
+        s.ngroups = 1;
+    } else {
+        s.ngroups = p.E + (p.S > 0 ? 1 : 0);
+    }
+    const int ng = s.ngroups;
+    for (int g = tid; g < ng; g += NTHREADS) {
+        int rows, row0;
+        if (p.offsets == nullptr) {
+            rows = p.T;
+            row0 = 0;
+        } else if (g < p.E) {
+            row0 = __ldg(p.offsets + g);
+            rows = __ldg(p.offsets + g + 1) - row0;
+            if (rows < 0 || row0 < 0 || row0 + rows > p.T * p.k) {
+                report_status(p.status, MS_ERR_DEVICE_INDEX);
+                rows = 0;
+            }
+        } else {
+            rows = p.T;
+            row0 = 0;
+        }
+        s.rows[g] = rows;
+        s.row0[g] = row0;
+        int units = 0;
+        if (rows > 0) {
+            if (Cfg<MODE>::kStream)
+                units = group_ntiles<MODE>(p, g) * group_ktiles<MODE>(p, g);
+            else
+                units = ((rows + BM - 1) / BM) * group_ntiles<MODE>(p, g);
+        }
+        s.prefix[g + 1] = units;   // scanned below
+    }
+    __syncthreads();
+    if (tid < 32) {
+        // inclusive scan over groups: each lane owns a run of groups
+        constexpr int kPer = (MAX_GROUPS + 31) / 32;
+        const int lane = tid;
+        int loc[kPer];
+        int sum = 0;
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int g = lane * kPer + q;
+            loc[q] = g < ng ? s.prefix[g + 1] : 0;
+            sum += loc[q];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int g = lane * kPer + q;
+            run += loc[q];
+            if (g < ng) s.prefix[g + 1] = run;
+        }
+        if (lane == 0) s.prefix[0] = 0;
+    }
+    __syncthreads();
+}
+
+// largest g with prefix[g] <= pos (g < ngroups); groups with no work have
+// prefix[g] == prefix[g+1] and are never returned for pos < total.
+__device__ __forceinline__ int find_group(const Sched& s, int pos) {
+    int lo = 0, hi = s.ngroups - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s.prefix[mid] <= pos) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+struct Seg {
+    int g, tile, k0, k1, kt, tile_start;   // tile: n-tile (streaming) / linear tile in group (tiled)
+};
+
+__device__ __forceinline__ long range_begin(int c, int total, int nct) {
+    return static_cast<long>(c) * total / nct;
+}
+// CTA whose range holds step `pos`: largest c with floor(c*total/nct) <= pos.
+__device__ __forceinline__ int cta_of(int pos, int total, int nct) {
+    const long num = static_cast<long>(pos + 1) * nct;
+    return static_cast<int>((num + total - 1) / total) - 1;
+}
+
+template <int MODE>
+__device__ __forceinline__ Seg stream_seg(const Params& p, const Sched& s, int pos, int end) {
+    Seg sg;
+    sg.g = find_group(s, pos);
+    sg.kt = group_ktiles<MODE>(p, sg.g);
+    const int local = pos - s.prefix[sg.g];
+    sg.tile = local / sg.kt;
+    sg.k0 = local - sg.tile * sg.kt;
+    sg.tile_start = pos - sg.k0;
+    const int left = end - pos;
+    sg.k1 = (sg.kt - sg.k0) < left ? sg.kt : sg.k0 + left;
+    return sg;
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// The epilogue's wait on an accumulator: one thread waits (bounded), the
+// named barrier hands its verdict to all 128 epilogue threads, so either all
+// of them go on or all of them stop -- none is left waiting at a barrier.
+__device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, uint64_t lim, volatile int* abort,
+                                         int etid, int& go) {
+    if (etid == 0) go = sm100::mbar_wait(bar, parity, lim, abort) ? 1 : 0;
+    epi_bar();
+    return *static_cast<volatile int*>(&go) != 0;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+// ------------------------------------------------------------ kernel
+template <int MODE, int NMAX>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
+    using L = Layout<MODE, NMAX>;
+    constexpr bool kStream = Cfg<MODE>::kStream;
+    constexpr bool kG1 = Cfg<MODE>::kG1;
+    constexpr int ST = L::STAGES;
+
+    extern __shared__ uint8_t dsmem[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t bar_full[ST], bar_empty[ST], bar_tfull[2], bar_tempty[2], bar_drain;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ volatile int abort_sh;
+    __shared__ int last_sh;
+    __shared__ int go_sh[2];
+    __shared__ Sched sched;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_addr(smem);
+
+    if (threadIdx.x == 0) {
+        tma_prefetch_map(&maps.w_a);
+        tma_prefetch_map(&maps.w_s);
+        tma_prefetch_map(&maps.tok_r);
+        tma_prefetch_map(&maps.tok_s);
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(smem_addr(&bar_full[i]), 1);
+            mbar_init(smem_addr(&bar_empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_addr(&bar_tfull[i]), 1);
+            mbar_init(smem_addr(&bar_tempty[i]), 4);
+        }
+        mbar_init(smem_addr(&bar_drain), 1);
+        abort_sh = 0;
+        fence_mbar_init();
+    }
+    // Everything below reads what earlier kernels wrote (routing offsets,
+    // gathered tokens, the previous GEMM's output) -- and TMEM is only taken
+    // once the previous kernel on the stream has finished with it.
+    grid_dep_wait();
+    if (warp == 1) {
+        tmem_alloc(smem_addr(&tmem_base_sh), TMEM_COLS);
+        tmem_relinquish();
+    }
+    build_schedule<MODE>(p, sched);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    grid_dep_launch();
+    const uint32_t tmem_base = tmem_base_sh;
+
+    const int total = sched.prefix[sched.ngroups];
+    const int nct = gridDim.x;
+    const int c = blockIdx.x;
+    // streaming: contiguous range of k-steps; tiled: tiles c, c+nct, ...
+    const int rb = kStream ? static_cast<int>(range_begin(c, total, nct)) : 0;
+    const int re = kStream ? static_cast<int>(range_begin(c + 1, total, nct)) : 0;
+    const uint64_t lim = p.wait_limit_ns;
+
+    if (warp == 0) {
+      if (lane == 0) {
+        // ---------------------------------------------------- TMA producer (one thread)
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t issued = 0, issued_par = 0;   // per stage: any load issued / its parity
+        bool ok = true;
+        auto produce_kstep = [&](int g, int tile, int kt, int rows, int row0, int m0) -> bool {
+            const bool shared = p.offsets != nullptr && g == p.E;
+            if (!mbar_wait(smem_addr(&bar_empty[stage]), phase ^ 1u, lim, &abort_sh)) return false;
+            const uint32_t full = smem_addr(&bar_full[stage]);
+            const uint32_t a = sbase + stage * L::STAGE;
+            const uint32_t b = a + L::A_BYTES;
+            {
+                const int kx = kt * BK;
+                if (kStream) {
+                    const int nb = (rows + TOKBOX - 1) / TOKBOX;
+                    mbar_expect_tx(full, L::A_BYTES + nb * TOKBOX * BK * 2);
+                    const int f0 = tile * BM;   // output-feature offset within the group
+                    if (MODE == G1_STREAM) {
+                        int z = g, fl = f0;
+                        const CUtensorMap* wm = &maps.w_a;
+                        if (shared) { z = f0 / p.I; fl = f0 - z * p.I; wm = &maps.w_s; }
+                        tma_load_3d(a, wm, full, kx, fl, z);
+                        tma_load_3d(a + TILE_BYTES, wm, full, kx, p.I + fl, z);
+                    } else if (MODE == G2_STREAM) {
+                        if (shared) {
+                            const int z = kx / p.I;
+                            tma_load_3d(a, &maps.w_s, full, kx - z * p.I, f0, z);
+                        } else {
+                            tma_load_3d(a, &maps.w_a, full, kx, f0, g);
+                        }
+                    } else {   // LM_STREAM
+                        tma_load_3d(a, &maps.w_a, full, kx, f0, 0);
+                    }
+                    const CUtensorMap* tm = shared ? &maps.tok_s : &maps.tok_r;
+                    for (int j = 0; j < nb; ++j)
+                        tma_load_3d(b + j * TOKBOX * BK * 2, tm, full, kx, row0 + j * TOKBOX, 0);
+                } else {
+                    mbar_expect_tx(full, L::A_BYTES + (MODE == G1_TILED ? 2 * TILE_BYTES : p.bn * BK * 2));
+                    const CUtensorMap* tm = shared ? &maps.tok_s : &maps.tok_r;
+                    tma_load_3d(a, tm, full, kx, row0 + m0, 0);
+                    if (MODE == G1_TILED) {
+                        const int f0 = tile * BM;
+                        int z = g, fl = f0;
+                        const CUtensorMap* wm = &maps.w_a;
+                        if (shared) { z = f0 / p.I; fl = f0 - z * p.I; wm = &maps.w_s; }
+                        tma_load_3d(b, wm, full, kx, fl, z);
+                        tma_load_3d(b + TILE_BYTES, wm, full, kx, p.I + fl, z);
+                    } else {
+                        const int n0 = tile * p.bn;
+                        for (int j = 0; j < p.bn / BM; ++j) {
+                            if (shared) {
+                                const int z = kx / p.I;
+                                tma_load_3d(b + j * TILE_BYTES, &maps.w_s, full, kx - z * p.I, n0 + j * BM, z);
+                            } else {
+                                tma_load_3d(b + j * TILE_BYTES, &maps.w_a, full, kx, n0 + j * BM, g);
+                            }
+                        }
+                    }
+                }
+            }
+            issued |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+            if (++stage == ST) { stage = 0; phase ^= 1u; }
+            return true;
+        };
+        if (kStream) {
+            for (int pos = rb; pos < re && ok;) {
+                const Seg sg = stream_seg<MODE>(p, sched, pos, re);
+                for (int kt = sg.k0; kt < sg.k1 && ok; ++kt)
+                    ok = produce_kstep(sg.g, sg.tile, kt, sched.rows[sg.g], sched.row0[sg.g], 0);
+                pos += sg.k1 - sg.k0;
+            }
+        } else {
+            for (int t = c; t < total && ok; t += nct) {
+                const int g = find_group(sched, t);
+                const int local = t - sched.prefix[g];
+                const int nt = group_ntiles<MODE>(p, g);
+                const int m = local / nt, n = local - m * nt;
+                const int kt_n = group_ktiles<MODE>(p, g);
+                for (int kt = 0; kt < kt_n && ok; ++kt)
+                    ok = produce_kstep(g, n, kt, sched.rows[g], sched.row0[g], m * BM);
+            }
+        }
+        if (!ok) {
+            report_status(p.status, MS_ERR_TIMEOUT);
+            abort_sh = 1;
+        }
+        // drain: every load this thread issued must land before the CTA exits
+        for (int s2 = 0; s2 < ST; ++s2)
+            if ((issued >> s2) & 1u) {
+                volatile int never = 0;
+                if (!mbar_wait(smem_addr(&bar_full[s2]), (issued_par >> s2) & 1u, lim, &never))
+                    report_status(p.status, MS_ERR_TIMEOUT);
+            }
+      }
+      __syncwarp();   // lanes 1..31 wait here so the warp reaches the final barrier converged
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ---------------------------------------------------- MMA issuer (one thread)
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        auto mma_tile = [&](int rows, int k0, int k1) -> bool {
+            if (!mbar_wait(smem_addr(&bar_tempty[acc]), acc_phase ^ 1u, lim, &abort_sh)) return false;
+            tc_fence_after();
+            uint32_t n_mma;
+            if (kStream) {
+                n_mma = static_cast<uint32_t>((rows + 15) / 16 * 16);
+            } else {
+                n_mma = MODE == G1_TILED ? 256u : static_cast<uint32_t>(p.bn);
+            }
+            const uint32_t idesc = idesc_bf16_f32(BM, n_mma);
+            const uint32_t d0 = tmem_base + acc * 256;
+            for (int kt = k0; kt < k1; ++kt) {
+                if (!mbar_wait(smem_addr(&bar_full[stage]), phase, lim, &abort_sh)) return false;
+                tc_fence_after();
+                {
+                    const uint32_t a = sbase + stage * L::STAGE;
+                    const uint32_t b = a + L::A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint32_t accum = (kt > k0 || kk > 0) ? 1u : 0u;
+                        const uint64_t bd = smem_desc_sw128(b + kk * 32);
+                        mma_bf16(d0, smem_desc_sw128(a + kk * 32), bd, idesc, accum);
+                        if (MODE == G1_STREAM)
+                            mma_bf16(d0 + 128, smem_desc_sw128(a + TILE_BYTES + kk * 32), bd, idesc, accum);
+                    }
+                    mma_commit(smem_addr(&bar_empty[stage]));
+                }
+                if (++stage == ST) { stage = 0; phase ^= 1u; }
+            }
+            mma_commit(smem_addr(&bar_tfull[acc]));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+            return true;
+        };
+        if (kStream) {
+            for (int pos = rb; pos < re && ok;) {
+                const Seg sg = stream_seg<MODE>(p, sched, pos, re);
+                ok = mma_tile(sched.rows[sg.g], sg.k0, sg.k1);
+                pos += sg.k1 - sg.k0;
+            }
+        } else {
+            for (int t = c; t < total && ok; t += nct) {
+                const int g = find_group(sched, t);
+                ok = mma_tile(sched.rows[g], 0, group_ktiles<MODE>(p, g));
+            }
+        }
+        if (!ok) {
+            report_status(p.status, MS_ERR_TIMEOUT);
+            abort_sh = 1;
+        }
+        // drain: all MMAs issued by this thread complete before TMEM is freed
+        mma_commit(smem_addr(&bar_drain));
+        volatile int never = 0;
+        if (!mbar_wait(smem_addr(&bar_drain), 0, lim, &never)) report_status(p.status, MS_ERR_TIMEOUT);
+      }
+      __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue (4 warps)
+        const int q = warp & 3;               // TMEM lane quadrant of this warp
+        const int r_in = q * 32 + lane;       // accumulator row held by this thread
+        const int etid = threadIdx.x - 64;    // 0..127
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        const int ldh_r = p.I, ldh_s = p.S * p.I;
+        auto tmem_at = [&](int col) -> uint32_t {
+            return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256 + col);
+        };
+        if (kStream) {
+            const int slot_floats = BM * NMAX * (kG1 ? 2 : 1);
+            for (int pos = rb; pos < re && ok;) {
+                const Seg sg = stream_seg<MODE>(p, sched, pos, re);
+                pos += sg.k1 - sg.k0;
+                if (!epi_wait(smem_addr(&bar_tfull[acc]), acc_phase, lim, &abort_sh, etid, go_sh[acc])) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int g = sg.g;
+                const bool shared = p.offsets != nullptr && g == p.E;
+                const int rows = sched.rows[g], row0 = sched.row0[g];
+                const int f = sg.tile * BM + r_in;       // output feature of this thread
+                const int nch = (rows + 15) / 16;
+                const bool whole = sg.k0 == 0 && sg.k1 == sg.kt;
+                float* my_slot = nullptr;
+                if (!whole) {
+                    const bool first = range_begin(c, total, nct) >= sg.tile_start;
+                    my_slot = p.partials + static_cast<size_t>(2 * c + (first ? 0 : 1)) * slot_floats;
+                }
+                for (int ch = 0; ch < nch; ++ch) {
+                    float va[16], vb[16];
+                    tmem_ld16(tmem_at(ch * 16), va);
+                    if (kG1) tmem_ld16(tmem_at(128 + ch * 16), vb);
+                    tmem_ld_wait();
+                    if (!whole) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            my_slot[(ch * 16 + j) * BM + r_in] = va[j];
+                            if (kG1) my_slot[(NMAX + ch * 16 + j) * BM + r_in] = vb[j];
+                        }
+                        continue;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = ch * 16 + j;
+                        if (t >= rows) break;
+                        if (MODE == G1_STREAM) {
+                            const float h = silu_mul(va[j], vb[j]);
+                            __nv_bfloat16* dst = shared ? p.h_sh + static_cast<size_t>(t) * ldh_s + f
+                                                        : p.h_perm + static_cast<size_t>(row0 + t) * ldh_r + f;
+                            *dst = __float2bfloat16_rn(h);
+                        } else if (MODE == G2_STREAM) {
+                            if (shared) {
+                                p.y_sh[static_cast<size_t>(t) * p.H + f] = va[j];
+                            } else if (p.y_bf16) {
+                                reinterpret_cast<__nv_bfloat16*>(p.y_perm)[static_cast<size_t>(row0 + t) * p.H + f] =
+                                    __float2bfloat16_rn(va[j]);
+                            } else {
+                                reinterpret_cast<float*>(p.y_perm)[static_cast<size_t>(row0 + t) * p.H + f] = va[j];
+                            }
+                        } else {
+                            p.logits[static_cast<size_t>(t) * p.V + f] = __float2bfloat16_rn(va[j]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&bar_tempty[acc]));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+                if (whole) continue;
+                // ---- split tile: the last contributor sums the partials in CTA order
+                const int c_first = cta_of(sg.tile_start, total, nct);
+                const int c_last = cta_of(sg.tile_start + sg.kt - 1, total, nct);
+                int nparts = 0;
+                for (int c2 = c_first; c2 <= c_last; ++c2)
+                    if (range_begin(c2 + 1, total, nct) > range_begin(c2, total, nct)) ++nparts;
+                int32_t* ctr = p.counters + static_cast<size_t>(g) * p.max_tiles + sg.tile;
+                __threadfence();
+                epi_bar();
+                if (etid == 0) {
+                    const int old = atomicAdd(ctr, 1);
+                    last_sh = (old == nparts - 1);
+                }
+                epi_bar();
+                if (!last_sh) continue;
+                __threadfence();
+                if (etid == 0) *ctr = 0;   // ready for the next call
+                for (int ch = 0; ch < nch; ++ch) {
+                    float va[16], vb[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) { va[j] = 0.f; vb[j] = 0.f; }
+                    for (int c2 = c_first; c2 <= c_last; ++c2) {
+                        const long b2 = range_begin(c2, total, nct);
+                        if (range_begin(c2 + 1, total, nct) <= b2) continue;
+                        const float* sl = p.partials +
+                                          static_cast<size_t>(2 * c2 + (b2 < sg.tile_start ? 1 : 0)) * slot_floats;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            va[j] += __ldcg(sl + (ch * 16 + j) * BM + r_in);
+                            if (kG1) vb[j] += __ldcg(sl + (NMAX + ch * 16 + j) * BM + r_in);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = ch * 16 + j;
+                        if (t >= rows) break;
+                        if (MODE == G1_STREAM) {
+                            const float h = silu_mul(va[j], vb[j]);
+                            __nv_bfloat16* dst = shared ? p.h_sh + static_cast<size_t>(t) * ldh_s + f
+                                                        : p.h_perm + static_cast<size_t>(row0 + t) * ldh_r + f;
+                            *dst = __float2bfloat16_rn(h);
+                        } else if (MODE == G2_STREAM) {
+                            if (shared) {
+                                p.y_sh[static_cast<size_t>(t) * p.H + f] = va[j];
+                            } else if (p.y_bf16) {
+                                reinterpret_cast<__nv_bfloat16*>(p.y_perm)[static_cast<size_t>(row0 + t) * p.H + f] =
+                                    __float2bfloat16_rn(va[j]);
+                            } else {
+                                reinterpret_cast<float*>(p.y_perm)[static_cast<size_t>(row0 + t) * p.H + f] = va[j];
+                            }
+                        } else {
+                            p.logits[static_cast<size_t>(t) * p.V + f] = __float2bfloat16_rn(va[j]);
+                        }
+                    }
+                }
+            }
+        } else {
+            for (int t = c; t < total && ok; t += nct) {
+                if (!epi_wait(smem_addr(&bar_tfull[acc]), acc_phase, lim, &abort_sh, etid, go_sh[acc])) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int g = find_group(sched, t);
+                const bool shared = p.offsets != nullptr && g == p.E;
+                const int local = t - sched.prefix[g];
+                const int nt = group_ntiles<MODE>(p, g);
+                const int m = local / nt, n = local - m * nt;
+                const int rr = m * BM + r_in;                 // row within the group
+                const bool valid = rr < sched.rows[g];
+                const size_t orow = static_cast<size_t>(shared ? rr : sched.row0[g] + rr);
+                if (MODE == G1_TILED) {
+                    const int f0 = n * BM;
+                    __nv_bfloat16* dst = shared ? p.h_sh + orow * ldh_s + f0 : p.h_perm + orow * ldh_r + f0;
+                    for (int ch = 0; ch < BM / 16; ++ch) {
+                        float g16[16], u16[16];
+                        tmem_ld16(tmem_at(ch * 16), g16);
+                        tmem_ld16(tmem_at(128 + ch * 16), u16);
+                        tmem_ld_wait();
+                        if (valid) {
+                            __align__(16) __nv_bfloat162 hb[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                hb[j] = __floats2bfloat162_rn(silu_mul(g16[2 * j], u16[2 * j]),
+                                                              silu_mul(g16[2 * j + 1], u16[2 * j + 1]));
+                            uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 16);
+                            d4[0] = reinterpret_cast<const uint4*>(hb)[0];
+                            d4[1] = reinterpret_cast<const uint4*>(hb)[1];
+                        }
+                    }
+                } else {
+                    const int n0 = n * p.bn;
+                    for (int ch = 0; ch < p.bn / 16; ++ch) {
+                        float v16[16];
+                        tmem_ld16(tmem_at(ch * 16), v16);
+                        tmem_ld_wait();
+                        if (!valid) continue;
+                        if (shared || !p.y_bf16) {
+                            float* dst = shared ? p.y_sh + orow * p.H + n0 + ch * 16
+                                                : reinterpret_cast<float*>(p.y_perm) + orow * p.H + n0 + ch * 16;
+                            float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                d4[j] = make_float4(v16[4 * j], v16[4 * j + 1], v16[4 * j + 2], v16[4 * j + 3]);
+                        } else {
+                            __align__(16) __nv_bfloat162 hb[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) hb[j] = __floats2bfloat162_rn(v16[2 * j], v16[2 * j + 1]);
+                            uint4* d4 = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.y_perm) +
+                                                                 orow * p.H + n0 + ch * 16);
+                            d4[0] = reinterpret_cast<const uint4*>(hb)[0];
+                            d4[1] = reinterpret_cast<const uint4*>(hb)[1];
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&bar_tempty[acc]));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+        }
+        if (!ok) {
+            if (etid == 0) report_status(p.status, MS_ERR_TIMEOUT);
+            abort_sh = 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// ------------------------------------------------------------ prep kernel
+// Gathers the routed token rows into expert order, pads token operands to
+// whole TMA boxes with zeros, and clears the split-tile counters.
+__global__ void __launch_bounds__(256) ffn_prep_kernel(const __nv_bfloat16* __restrict__ x,
+                                                       const int32_t* __restrict__ perm, int T,
+                                                       int H, int rows, int rows_pad,
+                                                       __nv_bfloat16* __restrict__ x_perm,
+                                                       __nv_bfloat16* __restrict__ x_pad,
+                                                       int t_pad, int32_t* __restrict__ ctr,
+                                                       int nctr, int32_t* status) {
+    grid_dep_wait();
+    grid_dep_launch();
+    const int n8 = H / 8;
+    const long stride = static_cast<long>(gridDim.x) * blockDim.x;
+    const long tid = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x;
+    const long n_perm = static_cast<long>(rows_pad) * n8;
+    for (long v = tid; v < n_perm; v += stride) {
+        const int r = static_cast<int>(v / n8), c = static_cast<int>(v % n8);
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (r < rows) {
+            const int t = __ldg(perm + r);
+            if (t >= 0 && t < T)
+                val = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H) + c);
+            else
+                report_status(status, MS_ERR_DEVICE_INDEX);
+        }
+        reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(r) * H)[c] = val;
+    }
+    if (x_pad) {
+        const long n_pad = static_cast<long>(t_pad) * n8;
+        for (long v = tid; v < n_pad; v += stride) {
+            const int r = static_cast<int>(v / n8), c = static_cast<int>(v % n8);
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (r < T) val = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * H) + c);
+            reinterpret_cast<uint4*>(x_pad + static_cast<size_t>(r) * H)[c] = val;
+        }
+    }
+    for (long v = tid; v < nctr; v += stride) ctr[v] = 0;
+}
+
+// ------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// bf16 tensor [d2][d1][d0] (d0 innermost), box {64, box_rows, 1}, 128-byte swizzle.
+// Every map is rank 3 (token operands use d2 = 1), so every load is the 3-D
+// form of cp.async.bulk.tensor: the instruction rank must match the map.
+static bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                     uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int MODE, int NMAX>
+static ms_status launch_gemm(int id, const Maps& maps, const Params& prm, cudaStream_t s) {
+    using L = Layout<MODE, NMAX>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE, NMAX>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+        if (e != cudaSuccess) {
+            set_cuda_error(e);
+            return MS_ERR_CUDA;
+        }
+        attr_set = true;
+    }
+    return launch(id, ffn_gemm_kernel<MODE, NMAX>, dim3(num_sms()), dim3(NTHREADS), L::SMEM, s, maps, prm);
+}
+
+template <int MODE>
+static ms_status launch_stream(int id, int nmax, const Maps& maps, const Params& prm, cudaStream_t s) {
+    switch (nmax) {
+        case 16: return launch_gemm<MODE, 16>(id, maps, prm, s);
+        case 32: return launch_gemm<MODE, 32>(id, maps, prm, s);
+        case 64: return launch_gemm<MODE, 64>(id, maps, prm, s);
+        default: return launch_gemm<MODE, 128>(id, maps, prm, s);
+    }
+}
+
+static int stream_nmax(int T) {
+    int n = 16;
+    while (n < T) n *= 2;
+    return n;
+}
+
+struct FfnWs {
+    int32_t* status;
+    __nv_bfloat16 *x_pad, *x_perm, *h_perm, *h_sh;
+    int32_t* counters;
+    float* partials;
+    size_t bytes;
+    int t_pad, rows_pad, max_tiles, nctr;
+};
+
+static FfnWs ffn_ws_layout(void* base, int T, int H, int E, int I, int S, int k) {
+    FfnWs w{};
+    char* p = static_cast<char*>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> char* {
+        char* r = p ? p + off : nullptr;
+        off += align_up(bytes, 1024);
+        return r;
+    };
+    const bool stream = T <= 128;
+    w.t_pad = static_cast<int>(align_up(T, BM));
+    w.rows_pad = static_cast<int>(align_up(static_cast<size_t>(T) * k, BM));
+    w.max_tiles = 1;
+    {
+        const int cand[3] = {(S > 0 ? S * I : I) / BM, H / BM, I / BM};
+        for (int q = 0; q < 3; ++q) w.max_tiles = cand[q] > w.max_tiles ? cand[q] : w.max_tiles;
+    }
+    const int ngroups = E + (S > 0 ? 1 : 0);
+    w.nctr = 2 * ngroups * w.max_tiles;
+    w.status = reinterpret_cast<int32_t*>(take(256));
+    w.x_pad = reinterpret_cast<__nv_bfloat16*>(take(stream ? static_cast<size_t>(w.t_pad) * H * 2 : 0));
+    w.x_perm = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(w.rows_pad) * H * 2));
+    w.h_perm = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(w.rows_pad) * I * 2));
+    w.h_sh = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(w.t_pad) * (S > 0 ? S * I : BK) * 2));
+    w.counters = reinterpret_cast<int32_t*>(take(static_cast<size_t>(w.nctr) * 4));
+    const size_t slot = static_cast<size_t>(BM) * (stream ? stream_nmax(T) : 16) * 2 * sizeof(float);
+    w.partials = reinterpret_cast<float*>(take(stream ? slot * 2 * num_sms() : 0));
+    w.bytes = off;
+    return w;
+}
+
+size_t ffn_ws_bytes(int T, int H, int E, int I, int S, int k) {
+    return ffn_ws_layout(nullptr, T, H, E, I, S, k).bytes;
+}
+
+ms_status ffn_launch(const void* x, const int32_t* offsets, const int32_t* perm, const void* wgu,
+                     const void* wd, const void* wsgu, const void* wsd, int T, int H, int E, int I,
+                     int S, int k, void* y_perm, ms_dtype ydt, float* y_sh, void* ws,
+                     cudaStream_t s) {
+    FfnWs w = ffn_ws_layout(ws, T, H, E, I, S, k);
+    const bool stream = T <= 128;
+    const int rows = T * k;
+    // 1. gather + pad + clear counters
+    {
+        const long work = static_cast<long>(w.rows_pad) * (H / 8);
+        const int grid = static_cast<int>(work / 256 + 1 < 4L * num_sms() ? work / 256 + 1 : 4L * num_sms());
+        ms_status st = launch(K_FFN_PREP, ffn_prep_kernel, dim3(grid), dim3(256), 0, s,
+                              reinterpret_cast<const __nv_bfloat16*>(x), perm, T, H, rows, w.rows_pad,
+                              w.x_perm, stream ? w.x_pad : static_cast<__nv_bfloat16*>(nullptr), w.t_pad,
+                              w.counters, w.nctr, w.status);
+        if (st != MS_OK) return st;
+    }
+    Params prm{};
+    prm.T = T; prm.H = H; prm.E = E; prm.I = I; prm.S = S; prm.k = k; prm.V = 0;
+    prm.bn = (H % 256 == 0) ? 256 : 128;
+    prm.offsets = offsets;
+    prm.h_perm = w.h_perm;
+    prm.h_sh = w.h_sh;
+    prm.y_perm = y_perm;
+    prm.y_bf16 = ydt == MS_BF16;
+    prm.y_sh = y_sh;
+    prm.partials = w.partials;
+    prm.status = w.status;
+    prm.max_tiles = w.max_tiles;
+    prm.wait_limit_ns = wait_limit_ns();
+    const int ngroups = E + (S > 0 ? 1 : 0);
+    const uint32_t tok_box = stream ? TOKBOX : BM;
+    const void* x_tok_s = stream ? static_cast<const void*>(w.x_pad) : x;
+    const int x_rows = stream ? w.t_pad : T;
+    // 2. GEMM1: gate/up + SwiGLU -> h
+    Maps m1{};
+    bool ok = make_map(&m1.w_a, wgu, H, 2 * I, E, BM) &&
+              make_map(&m1.tok_r, w.x_perm, H, w.rows_pad, 1, tok_box) &&
+              make_map(&m1.tok_s, x_tok_s, H, x_rows, 1, tok_box);
+    ok = ok && (S > 0 ? make_map(&m1.w_s, wsgu, H, 2 * I, S, BM) : make_map(&m1.w_s, wgu, H, 2 * I, E, BM));
+    if (!ok) return MS_ERR_CUDA;
+    prm.counters = w.counters;
+    ms_status st = stream ? launch_stream<G1_STREAM>(K_GEMM1_STREAM, stream_nmax(T), m1, prm, s)
+                          : launch_gemm<G1_TILED, 16>(K_GEMM1_TILED, m1, prm, s);
+    if (st != MS_OK) return st;
+    // 3. GEMM2: down projection -> y_perm, y_shared
+    Maps m2{};
+    const int hs_cols = S > 0 ? S * I : BK;
+    ok = make_map(&m2.w_a, wd, I, H, E, BM) && make_map(&m2.tok_r, w.h_perm, I, w.rows_pad, 1, tok_box) &&
+         make_map(&m2.tok_s, w.h_sh, hs_cols, w.t_pad, 1, tok_box);
+    ok = ok && (S > 0 ? make_map(&m2.w_s, wsd, I, H, S, BM) : make_map(&m2.w_s, wd, I, H, E, BM));
+    if (!ok) return MS_ERR_CUDA;
+    prm.counters = w.counters + ngroups * w.max_tiles;
+    return stream ? launch_stream<G2_STREAM>(K_GEMM2_STREAM, stream_nmax(T), m2, prm, s)
+                  : launch_gemm<G2_TILED, 16>(K_GEMM2_TILED, m2, prm, s);
+}
+
+// ------------------------------------------------------------ vocab head
+struct LmWs {
+    int32_t* status;
+    __nv_bfloat16* x_pad;
+    int32_t* counters;
+    float* partials;
+    size_t bytes;
+};
+
+static LmWs lm_ws_layout(void* base, int H, int V) {
+    LmWs w{};
+    char* p = static_cast<char*>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> char* {
+        char* r = p ? p + off : nullptr;
+        off += align_up(bytes, 1024);
+        return r;
+    };
+    w.status = reinterpret_cast<int32_t*>(take(256));
+    w.x_pad = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(BM) * H * 2));
+    w.counters = reinterpret_cast<int32_t*>(take(static_cast<size_t>(V / BM) * 4));
+    w.partials = reinterpret_cast<float*>(take(static_cast<size_t>(BM) * 128 * sizeof(float) * 2 * num_sms()));
+    w.bytes = off;
+    return w;
+}
+
+size_t lm_ws_bytes(int H, int V) { return lm_ws_layout(nullptr, H, V).bytes; }
+
+ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* logits, void* ws,
+                    cudaStream_t s) {
+    LmWs w = lm_ws_layout(ws, H, V);
+    for (int t0 = 0; t0 < T; t0 += BM) {
+        const int tc = T - t0 < BM ? T - t0 : BM;
+        const __nv_bfloat16* xc = reinterpret_cast<const __nv_bfloat16*>(x) + static_cast<size_t>(t0) * H;
+        ms_status st = launch(K_FFN_PREP, ffn_prep_kernel, dim3(2 * num_sms()), dim3(256), 0, s, xc,
+                              static_cast<const int32_t*>(nullptr), tc, H, 0, 0,
+                              static_cast<__nv_bfloat16*>(nullptr), w.x_pad, BM, w.counters, V / BM, w.status);
+        if (st != MS_OK) return st;
+        Maps m{};
+        bool ok = make_map(&m.w_a, wlm, H, V, 1, BM) && make_map(&m.w_s, wlm, H, V, 1, BM) &&
+                  make_map(&m.tok_r, w.x_pad, H, BM, 1, TOKBOX) && make_map(&m.tok_s, w.x_pad, H, BM, 1, TOKBOX);
+        if (!ok) return MS_ERR_CUDA;
+        Params prm{};
+        prm.T = tc; prm.H = H; prm.E = 1; prm.I = BM; prm.S = 0; prm.k = 1; prm.V = V;
+        prm.bn = 128;
+        prm.offsets = nullptr;
+        prm.logits = reinterpret_cast<__nv_bfloat16*>(logits) + static_cast<size_t>(t0) * V;
+        prm.partials = w.partials;
+        prm.counters = w.counters;
+        prm.status = w.status;
+        prm.max_tiles = V / BM;
+        prm.wait_limit_ns = wait_limit_ns();
+        st = launch_stream<LM_STREAM>(K_LM_HEAD, stream_nmax(tc), m, prm, s);
+        if (st != MS_OK) return st;
+    }
+    return MS_OK;
+}
+
+}  // namespace ms
+
+extern "C" size_t moe_expert_ffn_workspace_size(int T, int H, int E, int I, int S, int k) {
+    if (T <= 0 || H <= 0 || E <= 0 || I <= 0 || S < 0 || k <= 0) return 0;
+    return ms::ffn_ws_bytes(T, H, E, I, S, k);
+}
+
+extern "C" ms_status moe_expert_ffn(const void* xhat, const int32_t* expert_offsets,
+                                    const int32_t* perm_token, const void* w_gate_up,
+                                    const void* w_down, const void* ws_gate_up,
+                                    const void* ws_down, int T, int H, int E, int I, int S, int k,
+                                    void* y_perm, ms_dtype y_perm_dtype, float* y_shared, void* ws,
+                                    size_t ws_bytes, void* stream) {
+    if (!xhat || !expert_offsets || !perm_token || !w_gate_up || !w_down || !y_perm)
+        return MS_ERR_INVALID_ARG;
+    if (T <= 0 || H <= 0 || E <= 0 || I <= 0 || S < 0 || k <= 0 || k > E) return MS_ERR_INVALID_ARG;
+    if (y_perm_dtype != MS_F32 && y_perm_dtype != MS_BF16) return MS_ERR_INVALID_ARG;
+    if (S > 0 && (!ws_gate_up || !ws_down || !y_shared)) return MS_ERR_INVALID_ARG;
+    if (E > ms::MAX_GROUPS - 1 || H % 128 != 0 || I % 128 != 0 || S > 8) return MS_ERR_UNSUPPORTED;
+    if (static_cast<long>(T) * k > (1L << 30)) return MS_ERR_UNSUPPORTED;
+    if (!ms::aligned16(xhat) || !ms::aligned16(w_gate_up) || !ms::aligned16(w_down) || !ms::aligned16(y_perm) ||
+        (S > 0 && (!ms::aligned16(ws_gate_up) || !ms::aligned16(ws_down) || !ms::aligned16(y_shared))))
+        return MS_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < ms::ffn_ws_bytes(T, H, E, I, S, k)) return MS_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 1023u) return MS_ERR_INVALID_ARG;
+    // the status word at ws + 0 reports this call's device-side conditions only
+    cudaError_t ce = cudaMemsetAsync(ws, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
+    if (ce != cudaSuccess) {
+        ms::set_cuda_error(ce);
+        return MS_ERR_CUDA;
+    }
+    return ms::ffn_launch(xhat, expert_offsets, perm_token, w_gate_up, w_down, ws_gate_up, ws_down, T, H, E,
+                          I, S, k, y_perm, y_perm_dtype, y_shared, ws, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t lm_head_workspace_size(int T, int H, int V) {
+    if (T <= 0 || H <= 0 || V <= 0) return 0;
+    return ms::lm_ws_bytes(H, V);
+}
+
+extern "C" ms_status lm_head_logits(const void* xhat, const void* w_lm, int T, int H, int V,
+                                    void* logits_bf16, void* ws, size_t ws_bytes, void* stream) {
+    if (!xhat || !w_lm || !logits_bf16 || T <= 0 || H <= 0 || V <= 0) return MS_ERR_INVALID_ARG;
+    if (H % 128 != 0 || V % 128 != 0) return MS_ERR_UNSUPPORTED;
+    if (!ms::aligned16(xhat) || !ms::aligned16(w_lm) || !ms::aligned16(logits_bf16)) return MS_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < ms::lm_ws_bytes(H, V)) return MS_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 1023u) return MS_ERR_INVALID_ARG;
+    cudaError_t ce = cudaMemsetAsync(ws, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
+    if (ce != cudaSuccess) {
+        ms::set_cuda_error(ce);
+        return MS_ERR_CUDA;
+    }
+    return ms::lm_launch(xhat, w_lm, T, H, V, logits_bf16, ws, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,129 @@
+// Shared host/device helpers of libmoespec: launch with programmatic
+// dependent launch, tracing hooks, device status word, bounded waits.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <utility>
+
+#include "moespec.h"
+
+namespace ms {
+
+// ------------------------------------------------------------ kernel ids
+enum KernelId : int {
+    K_RMSNORM = 0,
+    K_ROUTE_ROWS,
+    K_ROUTE_TILED,
+    K_PERMUTE_COUNT,
+    K_PERMUTE_SCATTER,
+    K_FFN_PREP,
+    K_GEMM1_STREAM,
+    K_GEMM2_STREAM,
+    K_GEMM1_TILED,
+    K_GEMM2_TILED,
+    K_LM_HEAD,
+    K_COMBINE,
+    K_VERIFY_PARTIAL,
+    K_VERIFY_FINAL,
+    K_WAIT_PROBE,
+    K_COUNT
+};
+const char* kernel_name(int id);
+
+// ------------------------------------------------------------ host side
+void trace_mark(int id, cudaStream_t s, bool after);
+uint64_t wait_limit_ns();
+void set_cuda_error(cudaError_t e);
+
+// Launch `kernel` with programmatic stream serialisation allowed, so that it
+// may start while the previous kernel on the stream finishes; the kernel
+// itself calls grid_dep_wait() before touching dependent memory.
+template <typename... KArgs, typename... Args>
+inline ms_status launch(int id, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                        cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    trace_mark(id, s, false);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    trace_mark(id, s, true);
+    if (e != cudaSuccess) {
+        set_cuda_error(e);
+        return MS_ERR_CUDA;
+    }
+    return MS_OK;
+}
+
+inline int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------ device side
+// Wait for the kernel this one depends on (no-op when launched without PDL).
+__device__ __forceinline__ void grid_dep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Allow the next kernel on the stream to be scheduled.
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Record the first device-side error into a status word (first writer wins).
+__device__ __forceinline__ void report_status(int32_t* status, int32_t code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// Warp-wide (value, index) argmax step: larger value wins, equal values go
+// to the lower index.
+__device__ __forceinline__ void argmax_merge(float& v, int& i, float v2, int i2) {
+    if (v2 > v || (v2 == v && i2 < i)) {
+        v = v2;
+        i = i2;
+    }
+}
+
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+        int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+        argmax_merge(v, i, v2, i2);
+    }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+}  // namespace ms

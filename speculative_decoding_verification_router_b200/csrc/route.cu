@@ -1,0 +1,217 @@
+// a1: router logits (fp32), softmax over all experts and top-k selection.
+//
+// Top-6 of 64 routed experts (clawpit.io, "Lean architecture with a
+// compressed encoder").  Selection order: larger logit first, equal logits
+// to the lower expert index.  Gate weight = softmax probability of the
+// chosen expert (optionally renormalised over the k chosen).
+#include <math.h>
+
+#include "ms_common.cuh"
+
+namespace ms {
+
+constexpr int kMaxExperts = 256;
+
+// One warp: softmax over z[0..E) and the k best experts, written to
+// idx_out[0..k) / w_out[0..k).  Each lane holds experts lane, lane+32, ...
+__device__ void warp_topk_softmax(const float* z, int E, int k, int renorm, int32_t* idx_out,
+                                  float* w_out, int lane) {
+    constexpr int kPer = kMaxExperts / 32;
+    float v[kPer];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? z[e] : -INFINITY;
+        m = fmaxf(m, v[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+        if (lane + 32 * i < E) s += expf(v[i] - m);
+    s = warp_sum(s);
+    uint32_t taken = 0;
+    float wsum = 0.f;
+    float wsel = 0.f;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u)) argmax_merge(bv, bi, v[i], e);
+        }
+        warp_argmax(bv, bi);
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        const float p = expf(bv - m) / s;
+        wsum += p;
+        if (lane == j) wsel = p;
+        if (lane == 0) idx_out[j] = bi;
+    }
+    if (lane < k) w_out[lane] = renorm ? wsel / wsum : wsel;
+}
+
+// Small T: one block per token, 8 warps stride over experts; W_r rows are
+// read with float4 loads (L2-resident after the first token).
+__global__ void __launch_bounds__(256) route_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         const float* __restrict__ wr,
+                                                         const float* __restrict__ bias, int T,
+                                                         int H, int E, int k, int renorm,
+                                                         int32_t* __restrict__ idx,
+                                                         float* __restrict__ w) {
+    extern __shared__ float smem[];
+    float* xs = smem;       // [H]
+    float* z = smem + H;    // [E]
+    grid_dep_wait();
+    grid_dep_launch();
+    const int t = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+    for (int i = threadIdx.x; i < H / 8; i += blockDim.x) {
+        uint4 u = __ldg(xr + i);
+        const uint32_t p[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            xs[8 * i + 2 * q] = __uint_as_float(p[q] << 16);
+            xs[8 * i + 2 * q + 1] = __uint_as_float(p[q] & 0xffff0000u);
+        }
+    }
+    __syncthreads();
+    for (int e = warp; e < E; e += blockDim.x / 32) {
+        const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * H);
+        float acc = 0.f;
+        for (int h4 = lane; h4 < H / 4; h4 += 32) {
+            float4 a = __ldg(wrow + h4);
+            float4 b = *reinterpret_cast<const float4*>(xs + 4 * h4);
+            acc = fmaf(a.x, b.x, acc);
+            acc = fmaf(a.y, b.y, acc);
+            acc = fmaf(a.z, b.z, acc);
+            acc = fmaf(a.w, b.w, acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) z[e] = bias ? acc + __ldg(bias + static_cast<size_t>(t) * E + e) : acc;
+    }
+    __syncthreads();
+    if (warp == 0)
+        warp_topk_softmax(z, E, k, renorm, idx + static_cast<size_t>(t) * k,
+                          w + static_cast<size_t>(t) * k, lane);
+}
+
+// Large T (E <= 64): 64 tokens x 64 experts per block, register tile 4x4 per
+// thread, H walked in chunks of 32 through shared memory; then top-k per
+// token from the logits kept in shared memory.
+constexpr int RT_TOK = 64, RT_EXP = 64, RT_K = 32, RT_PAD = 4;
+
+__global__ void __launch_bounds__(256) route_tiled_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const float* __restrict__ wr,
+                                                          const float* __restrict__ bias, int T,
+                                                          int H, int E, int k, int renorm,
+                                                          int32_t* __restrict__ idx,
+                                                          float* __restrict__ w) {
+    __shared__ __align__(16) float xs[RT_K][RT_TOK + RT_PAD];
+    __shared__ __align__(16) float wsm[RT_K][RT_EXP + RT_PAD];
+    __shared__ float zs[RT_TOK][RT_EXP + 1];
+    grid_dep_wait();
+    grid_dep_launch();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t0 = blockIdx.x * RT_TOK;
+    const int ty = tid >> 4, tx = tid & 15;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+    const int lrow = tid >> 2;          // token (for x) / expert (for W) loaded by this thread
+    const int lseg = (tid & 3) * 8;     // 8 consecutive h
+    for (int h0 = 0; h0 < H; h0 += RT_K) {
+        {
+            const int t = t0 + lrow;
+            uint4 u = make_uint4(0, 0, 0, 0);
+            if (t < T)
+                u = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + h0 + lseg));
+            const uint32_t p[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                xs[lseg + 2 * q][lrow] = __uint_as_float(p[q] << 16);
+                xs[lseg + 2 * q + 1][lrow] = __uint_as_float(p[q] & 0xffff0000u);
+            }
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+            if (lrow < E) {
+                const float4* src = reinterpret_cast<const float4*>(wr + static_cast<size_t>(lrow) * H + h0 + lseg);
+                a = __ldg(src);
+                b = __ldg(src + 1);
+            }
+            wsm[lseg + 0][lrow] = a.x; wsm[lseg + 1][lrow] = a.y;
+            wsm[lseg + 2][lrow] = a.z; wsm[lseg + 3][lrow] = a.w;
+            wsm[lseg + 4][lrow] = b.x; wsm[lseg + 5][lrow] = b.y;
+            wsm[lseg + 6][lrow] = b.z; wsm[lseg + 7][lrow] = b.w;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < RT_K; ++kk) {
+            const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+            const float4 b = *reinterpret_cast<const float4*>(&wsm[kk][tx * 4]);
+            const float av[4] = {a.x, a.y, a.z, a.w};
+            const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = t0 + ty * 4 + i, e = tx * 4 + j;
+            float zv = acc[i][j];
+            if (bias && t < T && e < E) zv += __ldg(bias + static_cast<size_t>(t) * E + e);
+            zs[ty * 4 + i][e] = zv;
+        }
+    __syncthreads();
+    for (int r = warp; r < RT_TOK; r += 8) {
+        const int t = t0 + r;
+        if (t >= T) break;
+        warp_topk_softmax(zs[r], E, k, renorm, idx + static_cast<size_t>(t) * k,
+                          w + static_cast<size_t>(t) * k, lane);
+    }
+}
+
+ms_status route_launch(const void* x, const float* wr, const float* bias, int T, int H, int E,
+                       int k, int renorm, int32_t* idx, float* w, cudaStream_t s) {
+    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    if (T >= 1024 && E <= RT_EXP && H % RT_K == 0) {
+        dim3 grid((T + RT_TOK - 1) / RT_TOK);
+        return launch(K_ROUTE_TILED, route_tiled_kernel, grid, dim3(256), 0, s, xb, wr, bias, T, H,
+                      E, k, renorm, idx, w);
+    }
+    const size_t smem = sizeof(float) * static_cast<size_t>(H + E);
+    if (smem > 48 * 1024) {
+        static bool set = false;
+        if (!set) {
+            cudaFuncSetAttribute(route_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 200 * 1024);
+            set = true;
+        }
+    }
+    return launch(K_ROUTE_ROWS, route_rows_kernel, dim3(T), dim3(256), smem, s, xb, wr, bias, T,
+                  H, E, k, renorm, idx, w);
+}
+
+}  // namespace ms
+
+extern "C" ms_status moe_route_topk(const void* xhat, const float* w_router,
+                                    const float* logit_bias, int T, int H, int E, int k,
+                                    int renormalize, int32_t* topk_idx, float* topk_w,
+                                    void* stream) {
+    if (!xhat || !w_router || !topk_idx || !topk_w) return MS_ERR_INVALID_ARG;
+    if (T <= 0 || H <= 0 || E <= 0 || k <= 0 || k > E) return MS_ERR_INVALID_ARG;
+    if (E > ms::kMaxExperts || k > 32 || H % 128 != 0 || H > 48 * 1024) return MS_ERR_UNSUPPORTED;
+    if (!ms::aligned16(xhat) || !ms::aligned16(w_router)) return MS_ERR_INVALID_ARG;
+    return ms::route_launch(xhat, w_router, logit_bias, T, H, E, k, renormalize, topk_idx, topk_w,
+                            static_cast<cudaStream_t>(stream));
+}

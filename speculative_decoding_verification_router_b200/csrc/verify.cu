@@ -1,0 +1,196 @@
+// a6: greedy verification of one speculative step.
+//
+// The verifier picks its own greedy token at each of the K+1 positions,
+// accepts the longest prefix of drafts that agrees with those picks and
+// commits one more token of its own (jina.ai, "Modèle et entraînement";
+// clawpit.io, "Speculative decoding without accuracy loss"), so every step
+// commits between 1 and K+1 tokens.
+//
+// Kernel 1 splits every logits row into P chunks; each block streams its
+// chunk with 16-byte loads and reduces (max, lowest index).  Kernel 2, one
+// warp per sequence, merges the P partials per row and runs the prefix match.
+#include <math.h>
+
+#include "ms_common.cuh"
+
+namespace ms {
+
+constexpr int VF_THREADS = 256;
+constexpr int kMaxK = 8;
+
+__device__ __forceinline__ void vec_load(const float* p, float (&v)[4]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+__device__ __forceinline__ void vec_load(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(q[i] << 16);
+        v[2 * i + 1] = __uint_as_float(q[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ float scalar_load(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float scalar_load(const __nv_bfloat16* p) {
+    return bf16_to_f32(__ldg(reinterpret_cast<const uint16_t*>(p)));
+}
+
+template <typename TL>
+__global__ void __launch_bounds__(VF_THREADS) verify_partial_kernel(const TL* __restrict__ logits,
+                                                                    int V, int P, int chunk,
+                                                                    int vec_ok,
+                                                                    float* __restrict__ pv,
+                                                                    int32_t* __restrict__ pi) {
+    constexpr int VEC = 16 / sizeof(TL);
+    __shared__ float sv[VF_THREADS / 32];
+    __shared__ int si[VF_THREADS / 32];
+    grid_dep_wait();
+    grid_dep_launch();
+    const int r = blockIdx.x / P, p = blockIdx.x % P;
+    const int begin = p * chunk;
+    const int end = min(V, begin + chunk);
+    const TL* row = logits + static_cast<size_t>(r) * V;
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    int tail_begin = begin;
+    if (vec_ok) {
+        const int nvec = (end - begin) / VEC;
+        for (int q = threadIdx.x; q < nvec; q += VF_THREADS) {
+            float v[VEC];
+            const int i0 = begin + q * VEC;
+            vec_load(row + i0, v);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) argmax_merge(bv, bi, v[e], i0 + e);
+        }
+        tail_begin = begin + nvec * VEC;
+    }
+    for (int i = tail_begin + threadIdx.x; i < end; i += VF_THREADS)
+        argmax_merge(bv, bi, scalar_load(row + i), i);
+    warp_argmax(bv, bi);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) {
+        sv[warp] = bv;
+        si[warp] = bi;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        bv = lane < VF_THREADS / 32 ? sv[lane] : -INFINITY;
+        bi = lane < VF_THREADS / 32 ? si[lane] : 0x7fffffff;
+        warp_argmax(bv, bi);
+        if (lane == 0) {
+            pv[blockIdx.x] = bv;
+            pi[blockIdx.x] = bi;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(128) verify_final_kernel(const float* __restrict__ pv,
+                                                           const int32_t* __restrict__ pi, int B,
+                                                           int K, int P,
+                                                           const int32_t* __restrict__ draft,
+                                                           int32_t* __restrict__ argmax,
+                                                           int32_t* __restrict__ committed,
+                                                           int32_t* __restrict__ n_committed) {
+    grid_dep_wait();
+    grid_dep_launch();
+    const int b = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (b >= B) return;
+    int g[kMaxK + 1];
+#pragma unroll
+    for (int j = 0; j <= kMaxK; ++j) {
+        if (j > K) break;
+        const size_t base = (static_cast<size_t>(b) * (K + 1) + j) * P;
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int q = lane; q < P; q += 32) argmax_merge(bv, bi, pv[base + q], pi[base + q]);
+        warp_argmax(bv, bi);
+        g[j] = bi;
+    }
+    if (lane == 0) {
+        int n = 0;
+        while (n < K && __ldg(draft + static_cast<size_t>(b) * K + n) == g[n]) ++n;
+        int32_t* am = argmax + static_cast<size_t>(b) * (K + 1);
+        int32_t* cm = committed + static_cast<size_t>(b) * (K + 1);
+        for (int j = 0; j <= K; ++j) {
+            am[j] = g[j];
+            cm[j] = j < n ? g[j] : (j == n ? g[n] : -1);
+        }
+        n_committed[b] = n + 1;
+    }
+}
+
+struct VerifyPlan {
+    int P, chunk;
+};
+
+static VerifyPlan verify_plan(int B, int K, int V, int elem_bytes) {
+    const int rows = B * (K + 1);
+    const int vec = 16 / elem_bytes;
+    const int target = 4 * num_sms();
+    int P = (target + rows - 1) / rows;
+    const int maxP = (V + 1023) / 1024;
+    if (P > maxP) P = maxP;
+    if (P < 1) P = 1;
+    int chunk = (V + P - 1) / P;
+    chunk = (chunk + vec - 1) / vec * vec;
+    P = (V + chunk - 1) / chunk;
+    return {P, chunk};
+}
+
+size_t verify_ws_bytes(int B, int K, int V) {
+    // sized for the larger (fp32: more chunks) of the two element types
+    VerifyPlan p4 = verify_plan(B, K, V, 4), p2 = verify_plan(B, K, V, 2);
+    const int P = p4.P > p2.P ? p4.P : p2.P;
+    const size_t n = static_cast<size_t>(B) * (K + 1) * P;
+    return align_up(n * sizeof(float), 256) + align_up(n * sizeof(int32_t), 256);
+}
+
+ms_status verify_launch(const void* logits, ms_dtype dt, const int32_t* draft, int B, int K, int V,
+                        int32_t* argmax, int32_t* committed, int32_t* ncom, void* ws,
+                        cudaStream_t s) {
+    const int eb = dt == MS_BF16 ? 2 : 4;
+    const VerifyPlan plan = verify_plan(B, K, V, eb);
+    const int rows = B * (K + 1);
+    const size_t n = static_cast<size_t>(rows) * plan.P;
+    float* pv = static_cast<float*>(ws);
+    int32_t* pi = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align_up(n * sizeof(float), 256));
+    const int vec_ok = (V % (16 / eb) == 0) && aligned16(logits);
+    ms_status st;
+    if (dt == MS_BF16)
+        st = launch(K_VERIFY_PARTIAL, verify_partial_kernel<__nv_bfloat16>, dim3(rows * plan.P),
+                    dim3(VF_THREADS), 0, s, reinterpret_cast<const __nv_bfloat16*>(logits), V, plan.P,
+                    plan.chunk, vec_ok, pv, pi);
+    else
+        st = launch(K_VERIFY_PARTIAL, verify_partial_kernel<float>, dim3(rows * plan.P),
+                    dim3(VF_THREADS), 0, s, reinterpret_cast<const float*>(logits), V, plan.P,
+                    plan.chunk, vec_ok, pv, pi);
+    if (st != MS_OK) return st;
+    const int warps_per_block = 4;
+    return launch(K_VERIFY_FINAL, verify_final_kernel, dim3((B + warps_per_block - 1) / warps_per_block),
+                  dim3(32 * warps_per_block), 0, s, static_cast<const float*>(pv),
+                  static_cast<const int32_t*>(pi), B, K, plan.P, draft, argmax, committed, ncom);
+}
+
+}  // namespace ms
+
+extern "C" size_t spec_verify_workspace_size(int B, int K, int V) {
+    if (B <= 0 || K < 1 || V <= 0) return 0;
+    return ms::verify_ws_bytes(B, K, V);
+}
+
+extern "C" ms_status spec_verify_greedy(const void* logits, ms_dtype logits_dtype,
+                                        const int32_t* draft, int B, int K, int V,
+                                        int32_t* argmax, int32_t* committed,
+                                        int32_t* n_committed, void* ws, size_t ws_bytes,
+                                        void* stream) {
+    if (!logits || !draft || !argmax || !committed || !n_committed) return MS_ERR_INVALID_ARG;
+    if (B <= 0 || V <= 0 || K < 1) return MS_ERR_INVALID_ARG;
+    if (logits_dtype != MS_F32 && logits_dtype != MS_BF16) return MS_ERR_INVALID_ARG;
+    if (K > ms::kMaxK) return MS_ERR_UNSUPPORTED;
+    if (static_cast<long>(B) * (K + 1) * V > (1L << 40)) return MS_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < ms::verify_ws_bytes(B, K, V)) return MS_ERR_WORKSPACE;
+    return ms::verify_launch(logits, logits_dtype, draft, B, K, V, argmax, committed, n_committed,
+                             ws, static_cast<cudaStream_t>(stream));
+}
