@@ -290,8 +290,9 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     reps = max(1, (args.steps + steps_per_graph - 1) // steps_per_graph)
     steps = reps * steps_per_graph
-    for _ in range(2):
-        graph.replay()
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            graph.replay()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
@@ -300,10 +301,11 @@ def run_ours(args, rank, world, local):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    ev0.record(stream)
-    for _ in range(reps):
-        graph.replay()
-    ev1.record(stream)
+    with torch.cuda.stream(stream):          # replay on the stream the events time
+        ev0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        ev1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -313,19 +315,23 @@ def run_ours(args, rank, world, local):
     ms_per_step = elapsed_ms / steps
     value = aggregate_rate(prob.units_per_step() * steps, world, elapsed_ms / 1e3)
 
-    # per-kernel durations inside a traced run of the same steps (eager, same stream)
-    trace_steps = min(steps, 400)
+    # per-kernel durations: the library brackets every launch with CUDA events
+    # on the launching stream; the traced steps are captured in a CUDA graph so
+    # that host launch gaps do not enter the durations
+    trace_steps = steps_per_graph * max(1, 64 // steps_per_graph) if shp.layers == 1 else 2
     ms.trace_enable(per_step_launches * trace_steps + 16)
-    tev0, tev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    tev0.record(stream)
-    with torch.cuda.stream(stream):
+    tgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(tgraph, stream=stream):
         for i in range(trace_steps):
             prob.step(i)
-    tev1.record(stream)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        tgraph.replay()
     torch.cuda.synchronize()
     recs = ms.trace_records()
     ms.trace_disable()
     ms.trace_reset()
+    del tgraph
     per_kernel = {}
     for name, t in recs:
         per_kernel.setdefault(name, []).append(t)

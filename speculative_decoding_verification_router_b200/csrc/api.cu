@@ -50,19 +50,27 @@ static std::vector<TraceRec> g_recs;
 static int g_capacity = 0;
 static bool g_trace_on = false;
 
+// Inside stream capture an event must be recorded as an external record node,
+// otherwise it only orders work within the capture and never gets a timestamp.
+static void record(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &cs);
+    cudaEventRecordWithFlags(ev, s, cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                                        : cudaEventRecordDefault);
+}
+
 void trace_mark(int id, cudaStream_t s, bool after) {
     if (!g_trace_on) return;
     std::lock_guard<std::mutex> lk(g_trace_mu);
     if (!after) {
         if (static_cast<int>(g_recs.size()) >= g_capacity) return;
         TraceRec r{id, g_events[2 * g_recs.size()], g_events[2 * g_recs.size() + 1]};
-        cudaEventRecord(r.start, s);
+        record(r.start, s);
         g_recs.push_back(r);
     } else {
         if (g_recs.empty() || g_recs.back().id != id) return;
         // the matching stop is recorded once per start
-        TraceRec& r = g_recs.back();
-        cudaEventRecord(r.stop, s);
+        record(g_recs.back().stop, s);
     }
 }
 
