@@ -157,6 +157,26 @@ MS_API ms_status spec_verify_greedy(const void* logits, ms_dtype logits_dtype, c
                              int B, int K, int V, int32_t* argmax, int32_t* committed,
                              int32_t* n_committed, void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of spec_verify_greedy.  The pages have no
+ * counterpart: this exists for callers that cannot allocate device memory,
+ * e.g. a plugin running inside an inference server whose device memory is
+ * owned by the host application's pool, or a real-time decode loop that must
+ * not call cudaMalloc (which may synchronise the device) once it is running.
+ * Same arguments and results as spec_verify_greedy, minus (ws, ws_bytes):
+ * the partial maxima go to a static 128 KB device array inside the library,
+ * which every GPU that loads the library keeps until the process exits.
+ * Limit: batches whose partial maxima fit that array -- on a 148-SM B200 any
+ * batch with B*(K+1) <= 16384 rows; larger batches return MS_ERR_UNSUPPORTED
+ * and launch nothing.  The first call on each device looks the array's device
+ * address up (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture.  Every call uses the same array, so calls that may
+ * overlap on the GPU (other streams, other threads) race and must be ordered
+ * by the caller; nothing in it needs to start at zero.  Allocates nothing. */
+MS_API ms_status spec_verify_greedy_noalloc(const void* logits, ms_dtype logits_dtype,
+                                            const int32_t* draft, int B, int K, int V,
+                                            int32_t* argmax, int32_t* committed,
+                                            int32_t* n_committed, void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Whole layer in hot-path order: rmsnorm -> route -> permute -> expert FFN
  * -> combine.  a: [T,H] fp32 residual input, out: [T,H] fp32.  The

@@ -11,6 +11,8 @@
 // warp per sequence, merges the P partials per row and runs the prefix match.
 #include <math.h>
 
+#include <mutex>
+
 #include "ms_common.cuh"
 
 namespace ms {
@@ -173,7 +175,63 @@ ms_status verify_launch(const void* logits, ms_dtype dt, const int32_t* draft, i
                   static_cast<const int32_t*>(pi), B, K, plan.P, draft, argmax, committed, ncom);
 }
 
+// ---------------------------------------------------------------- no-alloc
+// Scratch for spec_verify_greedy_noalloc: the per-chunk partial maxima live in
+// this file-scope device array instead of a caller workspace.  Every GPU that
+// loads the library holds these 128 KB (plus alignment slack) until the
+// process exits.  16,384 partial entries cover every batch of up to 16,384
+// verify rows (B*(K+1)) on a 148-SM B200.
+constexpr size_t kNoAllocScratchBytes = 2 * 16384 * sizeof(float) + 256;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Host code cannot use `g_noalloc_scratch` as a pointer: in host code the name
+// stands for a host-side shadow, not the device address.  The device address is
+// looked up once per device, with that device current, and cached.
+static ms_status noalloc_scratch(void** out) {
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_cuda_error(e);
+        return MS_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= 64) return MS_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) {
+            set_cuda_error(e);
+            return MS_ERR_CUDA;
+        }
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return MS_OK;
+}
+
 }  // namespace ms
+
+// Greedy verification without a caller workspace, for callers that cannot
+// allocate device memory (see include/moespec.h).
+extern "C" ms_status spec_verify_greedy_noalloc(const void* logits, ms_dtype logits_dtype,
+                                                const int32_t* draft, int B, int K, int V,
+                                                int32_t* argmax, int32_t* committed,
+                                                int32_t* n_committed, void* stream) {
+    if (!logits || !draft || !argmax || !committed || !n_committed) return MS_ERR_INVALID_ARG;
+    if (B <= 0 || V <= 0 || K < 1) return MS_ERR_INVALID_ARG;
+    if (logits_dtype != MS_F32 && logits_dtype != MS_BF16) return MS_ERR_INVALID_ARG;
+    if (K > ms::kMaxK) return MS_ERR_UNSUPPORTED;
+    if (static_cast<long>(B) * (K + 1) * V > (1L << 40)) return MS_ERR_UNSUPPORTED;
+    // the partial maxima of this batch must fit the static scratch
+    if (ms::verify_ws_bytes(B, K, V) > ms::kNoAllocScratchBytes) return MS_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    ms_status st = ms::noalloc_scratch(&scratch);
+    if (st != MS_OK) return st;
+    return ms::verify_launch(logits, logits_dtype, draft, B, K, V, argmax, committed, n_committed, scratch,
+                             static_cast<cudaStream_t>(stream));
+}
 
 extern "C" size_t spec_verify_workspace_size(int B, int K, int V) {
     if (B <= 0 || K < 1 || V <= 0) return 0;
