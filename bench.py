@@ -163,11 +163,13 @@ class Problem:
         self.n_sets = n_sets
         self.layers = []
         for _ in range(n_sets):
+            # weights are repacked once, at load time, into the GEMMs' tile layout
+            pk = lambda t: ms.pack_weights(t)
             self.layers.append(dict(
-                wgu=randn((E, 2 * I, H), shp.weight_std, torch.bfloat16),
-                wd=randn((E, H, I), shp.weight_std, torch.bfloat16),
-                wsgu=randn((S, 2 * I, H), shp.weight_std, torch.bfloat16),
-                wsd=randn((S, H, I), shp.weight_std, torch.bfloat16),
+                wgu=pk(randn((E, 2 * I, H), shp.weight_std, torch.bfloat16)),
+                wd=pk(randn((E, H, I), shp.weight_std, torch.bfloat16)),
+                wsgu=pk(randn((S, 2 * I, H), shp.weight_std, torch.bfloat16)),
+                wsd=pk(randn((S, H, I), shp.weight_std, torch.bfloat16)),
                 wr=randn((E, H), shp.router_std, torch.float32)))
         b = synth.router_bias(shp, seed)
         self.bias = None if b is None else torch.from_numpy(b).to(device)
@@ -177,7 +179,7 @@ class Problem:
         self.verify = shp.K > 0
         if self.verify:
             B, K, V = shp.B, shp.K, shp.V
-            self.lm = randn((V, H), shp.weight_std, torch.bfloat16) if shp.layers > 1 else None
+            self.lm = ms.pack_weights(randn((V, H), shp.weight_std, torch.bfloat16)) if shp.layers > 1 else None
             self.n_logit_sets = 1 if self.lm is not None else max(n_sets, 1)
             self.logits = [randn((B, K + 1, V), 1.0, torch.bfloat16) if self.lm is None
                            else torch.empty((T, V), dtype=torch.bfloat16, device=device)

@@ -101,7 +101,18 @@ MS_API ms_status moe_permute(const int32_t* topk_idx, int T, int k, int E,
                       int32_t* expert_offsets, int32_t* perm_token, int32_t* slot_of,
                       void* ws, size_t ws_bytes, void* stream);
 
+/* Weight layout for the tensor-core GEMMs.  A bf16 matrix stack W[n][rows][cols]
+ * (cols = the contraction dimension) is repacked once, at load time, into
+ * P[n][rows/128][cols/64][128][64]: each 128-row x 64-column tile the GEMMs
+ * load is one contiguous 16 KB block, so weight streaming reads whole DRAM
+ * pages.  Values are unchanged.  rows % 128 == 0, cols % 64 == 0; w and packed
+ * are distinct device buffers of n*rows*cols bf16 each.  The pages do not
+ * describe storage; this is the library's own format. */
+MS_API ms_status moe_pack_weights(const void* w, int n, int rows, int cols, void* packed, void* stream);
+
 /* a3  Expert FFN: every routed row and the shared experts, SwiGLU.
+ * All four weight arguments are in the packed layout of moe_pack_weights
+ * (w_gate_up: n=E, rows=2I, cols=H; w_down: n=E, rows=H, cols=I; shared: n=S).
  * For grouped row r of expert e (token t = perm_token[r]):
  *   g = W_g[e] x_t, u = W_u[e] x_t, h = silu(g) * u (rounded to bf16),
  *   y_perm[r,:] = W_d[e] h            (fp32 accumulation throughout)
@@ -132,7 +143,8 @@ MS_API ms_status moe_combine(const void* y_perm, ms_dtype y_perm_dtype, const fl
                       int T, int H, int k, float* out, void* out_bf16, void* stream);
 
 /* a5  Vocab head for the verify rows: logits[t,v] = sum_h xhat[t,h] w_lm[v,h].
- * xhat: [T,H] bf16, w_lm: [V,H] bf16, logits: [T,V] bf16 (fp32 accumulate).
+ * xhat: [T,H] bf16, w_lm: [V,H] bf16 packed by moe_pack_weights (n=1, rows=V,
+ * cols=H), logits: [T,V] bf16 (fp32 accumulate).
  * V % 128 == 0.  Tensor-core GEMM; T is processed 128 rows at a time.
  * Scratch: lm_head_workspace_size(T,H,V) bytes. */
 MS_API size_t lm_head_workspace_size(int T, int H, int V);
@@ -179,8 +191,9 @@ MS_API ms_status spec_verify_greedy_noalloc(const void* logits, ms_dtype logits_
 
 /* ---------------------------------------------------------------------- */
 /* Whole layer in hot-path order: rmsnorm -> route -> permute -> expert FFN
- * -> combine.  a: [T,H] fp32 residual input, out: [T,H] fp32.  The
- * intermediates live in ws (moe_layer_workspace_size bytes). */
+ * -> combine.  a: [T,H] fp32 residual input, out: [T,H] fp32.  Expert weights
+ * as for moe_expert_ffn (packed).  The intermediates live in ws
+ * (moe_layer_workspace_size bytes). */
 MS_API size_t moe_layer_workspace_size(int T, int H, int E, int I, int S, int k);
 MS_API ms_status moe_layer_forward(const float* a, const float* w_router, const float* logit_bias,
                             const void* w_gate_up, const void* w_down,
@@ -206,6 +219,16 @@ MS_API uint64_t ms_get_wait_limit_ns(void);
  * (device int32).  flag, status: device pointers. */
 MS_API ms_status ms_debug_bounded_wait(const int32_t* flag, int32_t expect, int32_t* status,
                                 void* stream);
+
+/* In-kernel timeline of the tensor-core GEMMs: while a device buffer of at
+ * least 5*256*8 uint64 (80 KB) is set, every CTA of every GEMM launch writes
+ * globaltimer stamps (ns) to buf[(mode*256 + cta)*8 + slot], mode 0..4 =
+ * GEMM1 streaming, GEMM2 streaming, vocab head, GEMM1 tiled, GEMM2 tiled;
+ * slot 0 entry, 1 schedule built, 2 setup done (after the wait on the previous
+ * kernel), 3 first stage of data ready, 4 last MMA issued, 5 epilogue done,
+ * 6 loads drained, 7 exit.  A later launch of the same mode overwrites.
+ * buf = NULL disables it.  For profiling only. */
+MS_API ms_status ms_set_device_trace(void* buf, size_t bytes);
 
 /* Launch tracing: when enabled, every kernel this library launches is
  * bracketed by a pair of CUDA events (recorded on the launching stream, so

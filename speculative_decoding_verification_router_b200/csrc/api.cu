@@ -13,6 +13,8 @@ namespace ms {
 ms_status rmsnorm_launch(const float*, const float*, int, int, float, void*, cudaStream_t);
 ms_status route_launch(const void*, const float*, const float*, int, int, int, int, int, int32_t*,
                        float*, cudaStream_t);
+ms_status route_cluster_launch(const void*, bool, float, const float*, const float*, int, int, int, int, int,
+                               int32_t*, float*, void*, cudaStream_t);
 size_t permute_ws_bytes(int, int, int);
 ms_status permute_launch(const int32_t*, int, int, int, int32_t*, int32_t*, int32_t*, void*, int32_t*,
                          cudaStream_t);
@@ -21,11 +23,13 @@ ms_status ffn_launch(const void*, const int32_t*, const int32_t*, const void*, c
                      const void*, int, int, int, int, int, int, void*, ms_dtype, float*, void*, cudaStream_t);
 ms_status combine_launch(const void*, ms_dtype, const float*, const int32_t*, const float*, const float*,
                          int, int, int, float*, void*, cudaStream_t);
+void set_device_trace(void*);
 
 static const char* kNames[K_COUNT] = {
-    "rmsnorm",        "route_rows",      "route_tiled",     "permute_count", "permute_scatter",
+    "rmsnorm",        "route_rows",      "route_tiled",     "route_cluster", "permute_count", "permute_scatter",
     "ffn_prep",       "gemm1_stream",    "gemm2_stream",    "gemm1_tiled",   "gemm2_tiled",
-    "lm_head_stream", "combine",         "verify_partial",  "verify_final",  "wait_probe"};
+    "lm_head_stream", "combine",         "verify_partial",  "verify_final",  "verify_cluster", "wait_probe",
+    "pack_weights"};
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kNames[id] : "?"; }
 
@@ -156,9 +160,16 @@ ms_status moe_layer_forward(const float* a, const float* w_router, const float* 
         ms::set_cuda_error(ce);
         return MS_ERR_CUDA;
     }
-    ms_status st = ms::rmsnorm_launch(a, nullptr, T, H, 1e-6f, w.xhat, s);
-    if (st == MS_OK)
-        st = ms::route_launch(w.xhat, w_router, logit_bias, T, H, E, k, renormalize, w.idx, w.w, s);
+    ms_status st;
+    if (T < 1024) {
+        // normalisation fused into the router's clusters
+        st = ms::route_cluster_launch(a, true, 1e-6f, w_router, logit_bias, T, H, E, k, renormalize, w.idx, w.w,
+                                      w.xhat, s);
+    } else {
+        st = ms::rmsnorm_launch(a, nullptr, T, H, 1e-6f, w.xhat, s);
+        if (st == MS_OK)
+            st = ms::route_launch(w.xhat, w_router, logit_bias, T, H, E, k, renormalize, w.idx, w.w, s);
+    }
     if (st == MS_OK) st = ms::permute_launch(w.idx, T, k, E, w.offsets, w.perm, w.slot, w.perm_ws, status, s);
     if (st == MS_OK)
         st = ms::ffn_launch(w.xhat, w.offsets, w.perm, w_gate_up, w_down, ws_gate_up, ws_down, T, H, E, I, S, k,
@@ -184,6 +195,12 @@ ms_status ms_device_status(void* ws, void* stream) {
 }
 
 void ms_set_wait_limit_ns(uint64_t ns) { ms::g_wait_limit_ns = ns; }
+
+ms_status ms_set_device_trace(void* buf, size_t bytes) {
+    if (buf && bytes < static_cast<size_t>(5) * 256 * 8 * sizeof(uint64_t)) return MS_ERR_WORKSPACE;
+    ms::set_device_trace(buf);
+    return MS_OK;
+}
 uint64_t ms_get_wait_limit_ns(void) { return ms::g_wait_limit_ns; }
 
 ms_status ms_debug_bounded_wait(const int32_t* flag, int32_t expect, int32_t* status, void* stream) {

@@ -66,7 +66,14 @@ struct Params {
     int32_t* status;
     int max_tiles;                 // tiles per group upper bound (counter stride)
     uint64_t wait_limit_ns;
+    uint64_t* dtrace;              // optional per-CTA timeline (see ms_set_device_trace)
 };
+
+// Timeline slots written per CTA when a device trace buffer is set.
+enum TraceSlot { TS_ENTRY = 0, TS_SCHEDULE, TS_SETUP, TS_FIRST_DATA, TS_LAST_MMA, TS_EPI_DONE, TS_PRODUCER_DONE, TS_EXIT };
+__device__ __forceinline__ void tstamp(const Params& p, int mode, int slot) {
+    if (p.dtrace) p.dtrace[(static_cast<size_t>(mode) * 256 + blockIdx.x) * 8 + slot] = global_ns();
+}
 
 template <int MODE>
 struct Cfg {
@@ -215,6 +222,87 @@ __device__ __forceinline__ Seg stream_seg(const Params& p, const Sched& s, int p
     return sg;
 }
 
+// ------------------------------------------------------------ work order
+// One unit of work = the k-steps [k0, k1) of one output tile, accumulated into
+// one TMEM buffer.  All three roles walk the same sequence.
+struct Work {
+    int g, n, m0, k0, k1, kt, tile_start;
+};
+
+template <int MODE>
+struct WorkIter {
+    // streaming: this CTA's contiguous k-step range [rb, re), visited in the
+    // order [split tile at the end of the range], then [rb, last_start): the
+    // tiles shared with a neighbour CTA come first, so their fix-up overlaps
+    // the streaming of the whole tiles instead of forming the kernel's tail.
+    // tiled: tiles c, c + nct, ...
+    int rb, re, last_start, pos, state, t, total, nct;
+
+    __device__ void init(const Params& p, const Sched& s, int c, int nct_) {
+        nct = nct_;
+        total = s.prefix[s.ngroups];
+        if (Cfg<MODE>::kStream) {
+            rb = static_cast<int>(range_begin(c, total, nct));
+            re = static_cast<int>(range_begin(c + 1, total, nct));
+            state = 0;
+            if (re > rb) {
+                const int g = find_group(s, re - 1);
+                const int kt = group_ktiles<MODE>(p, g);
+                const int local = re - 1 - s.prefix[g];
+                const int ts = re - 1 - (local % kt);
+                last_start = ts > rb ? ts : rb;
+            } else {
+                last_start = rb;
+                state = 2;
+            }
+        } else {
+            t = c;
+        }
+    }
+
+    __device__ bool next(const Params& p, const Sched& s, Work& w) {
+        if (Cfg<MODE>::kStream) {
+            int from, to;
+            if (state == 0) {
+                from = last_start;
+                to = re;
+                state = 1;
+                pos = rb;
+            } else if (state == 1 && pos < last_start) {
+                from = pos;
+                to = last_start;
+            } else {
+                return false;
+            }
+            const Seg sg = stream_seg<MODE>(p, s, from, to);
+            if (state == 1 && from != last_start) pos = from + (sg.k1 - sg.k0);
+            w.g = sg.g;
+            w.n = sg.tile;
+            w.m0 = 0;
+            w.k0 = sg.k0;
+            w.k1 = sg.k1;
+            w.kt = sg.kt;
+            w.tile_start = sg.tile_start;
+            return true;
+        } else {
+            if (t >= total) return false;
+            const int g = find_group(s, t);
+            const int local = t - s.prefix[g];
+            const int nt = group_ntiles<MODE>(p, g);
+            const int m = local / nt;
+            w.g = g;
+            w.n = local - m * nt;
+            w.m0 = m * BM;
+            w.k0 = 0;
+            w.kt = group_ktiles<MODE>(p, g);
+            w.k1 = w.kt;
+            w.tile_start = -1;
+            t += nct;
+            return true;
+        }
+    }
+};
+
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // The epilogue's wait on an accumulator: one thread waits (bounded), the
@@ -228,6 +316,10 @@ __device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, uint64_t
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+// Row of the packed weight tensor (see pack.cu) that starts the 128-row x
+// 64-column tile at (row r0, k-step kb) of a matrix with `kt` k-steps per row.
+__device__ __forceinline__ int packed_row(int r0, int kb, int kt) { return ((r0 / BM) * kt + kb) * BM; }
 
 // ------------------------------------------------------------ kernel
 template <int MODE, int NMAX>
@@ -249,8 +341,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t sbase = smem_addr(smem);
+    const int c = blockIdx.x, nct = gridDim.x;
+    const uint64_t lim = p.wait_limit_ns;
 
     if (threadIdx.x == 0) {
+        tstamp(p, MODE, TS_ENTRY);
         tma_prefetch_map(&maps.w_a);
         tma_prefetch_map(&maps.w_s);
         tma_prefetch_map(&maps.tok_r);
@@ -267,185 +362,190 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         abort_sh = 0;
         fence_mbar_init();
     }
-    // Everything below reads what earlier kernels wrote (routing offsets,
-    // gathered tokens, the previous GEMM's output) -- and TMEM is only taken
-    // once the previous kernel on the stream has finished with it.
+    // The schedule needs only the routing offsets.  They were written two
+    // kernels back on this stream (the permutation, before the gather kernel
+    // or GEMM1 that precedes this launch); that predecessor already waited
+    // for them, so they are complete even while it is still running.
+    build_schedule<MODE>(p, sched);
+    if (threadIdx.x == 0) tstamp(p, MODE, TS_SCHEDULE);
+
+    // ---- producer state (thread 0), kept across the dependency wait
+    const int kt_h = p.H / BK, kt_i = p.I / BK;
+    int q_issued = 0;                       // k-steps whose loads were issued
+    int npre = 0;                           // k-steps whose weight half was prefetched
+    auto weight_loads = [&](const Work& w, int kt, uint32_t a, uint32_t b, uint32_t full) {
+        const bool shared = p.offsets != nullptr && w.g == p.E;
+        const int kx = kt * BK;
+        if (MODE == G1_STREAM || MODE == G1_TILED) {
+            int z = w.g, fl = w.n * BM;
+            const CUtensorMap* wm = &maps.w_a;
+            if (shared) { z = fl / p.I; fl -= z * p.I; wm = &maps.w_s; }
+            const uint32_t dst = MODE == G1_STREAM ? a : b;
+            tma_load_3d(dst, wm, full, 0, packed_row(fl, kt, kt_h), z);
+            tma_load_3d(dst + TILE_BYTES, wm, full, 0, packed_row(p.I + fl, kt, kt_h), z);
+        } else if (MODE == G2_STREAM) {
+            const int f0 = w.n * BM;
+            if (shared) {
+                const int z = kx / p.I;
+                tma_load_3d(a, &maps.w_s, full, 0, packed_row(f0, (kx - z * p.I) / BK, kt_i), z);
+            } else {
+                tma_load_3d(a, &maps.w_a, full, 0, packed_row(f0, kt, kt_i), w.g);
+            }
+        } else if (MODE == LM_STREAM) {
+            tma_load_3d(a, &maps.w_a, full, 0, packed_row(w.n * BM, kt, kt_h), 0);
+        } else {   // G2_TILED
+            const int n0 = w.n * p.bn;
+            for (int j = 0; j < p.bn / BM; ++j) {
+                if (shared) {
+                    const int z = kx / p.I;
+                    tma_load_3d(b + j * TILE_BYTES, &maps.w_s, full, 0,
+                                packed_row(n0 + j * BM, (kx - z * p.I) / BK, kt_i), z);
+                } else {
+                    tma_load_3d(b + j * TILE_BYTES, &maps.w_a, full, 0, packed_row(n0 + j * BM, kt, kt_i), w.g);
+                }
+            }
+        }
+    };
+    auto weight_bytes = [&]() -> uint32_t {
+        if (MODE == G1_STREAM || MODE == G1_TILED) return 2 * TILE_BYTES;
+        if (MODE == G2_TILED) return p.bn * BK * 2;
+        return TILE_BYTES;
+    };
+    auto token_loads = [&](const Work& w, int kt, uint32_t a, uint32_t b, uint32_t full) -> uint32_t {
+        const bool shared = p.offsets != nullptr && w.g == p.E;
+        const CUtensorMap* tm = shared ? &maps.tok_s : &maps.tok_r;
+        const int row0 = sched.row0[w.g];
+        if (kStream) {
+            const int nb = (sched.rows[w.g] + TOKBOX - 1) / TOKBOX;
+            mbar_expect_tx(full, nb * TOKBOX * BK * 2);
+            for (int j = 0; j < nb; ++j) tma_load_3d(b + j * TOKBOX * BK * 2, tm, full, kt * BK, row0 + j * TOKBOX, 0);
+        } else {
+            mbar_expect_tx(full, TILE_BYTES);
+            tma_load_3d(a, tm, full, kt * BK, row0 + w.m0, 0);
+        }
+        return 0;
+    };
+
+    if (threadIdx.x == 0) {
+        // Weight tiles do not depend on the previous kernel: start streaming
+        // the first stages now, while it drains.
+        WorkIter<MODE> it;
+        it.init(p, sched, c, nct);
+        Work w;
+        while (npre < ST && it.next(p, sched, w)) {
+            for (int kt = w.k0; kt < w.k1 && npre < ST; ++kt, ++npre) {
+                const uint32_t a = sbase + npre * L::STAGE, full = smem_addr(&bar_full[npre]);
+                mbar_expect_tx_only(full, weight_bytes());
+                weight_loads(w, kt, a, a + L::A_BYTES, full);
+            }
+        }
+    }
+
+    // Everything below may read what the previous kernels wrote (gathered
+    // tokens, the previous GEMM's output) or overwrite what they still read,
+    // and TMEM is only taken once the previous kernel has released it.
     grid_dep_wait();
     if (warp == 1) {
         tmem_alloc(smem_addr(&tmem_base_sh), TMEM_COLS);
         tmem_relinquish();
     }
-    build_schedule<MODE>(p, sched);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     grid_dep_launch();
     const uint32_t tmem_base = tmem_base_sh;
-
-    const int total = sched.prefix[sched.ngroups];
-    const int nct = gridDim.x;
-    const int c = blockIdx.x;
-    // streaming: contiguous range of k-steps; tiled: tiles c, c+nct, ...
-    const int rb = kStream ? static_cast<int>(range_begin(c, total, nct)) : 0;
-    const int re = kStream ? static_cast<int>(range_begin(c + 1, total, nct)) : 0;
-    const uint64_t lim = p.wait_limit_ns;
+    if (threadIdx.x == 0) tstamp(p, MODE, TS_SETUP);
 
     if (warp == 0) {
       if (lane == 0) {
         // ---------------------------------------------------- TMA producer (one thread)
-        int stage = 0;
-        uint32_t phase = 0;
-        uint32_t issued = 0, issued_par = 0;   // per stage: any load issued / its parity
         bool ok = true;
-        auto produce_kstep = [&](int g, int tile, int kt, int rows, int row0, int m0) -> bool {
-            const bool shared = p.offsets != nullptr && g == p.E;
-            if (!mbar_wait(smem_addr(&bar_empty[stage]), phase ^ 1u, lim, &abort_sh)) return false;
-            const uint32_t full = smem_addr(&bar_full[stage]);
-            const uint32_t a = sbase + stage * L::STAGE;
-            const uint32_t b = a + L::A_BYTES;
-            {
-                const int kx = kt * BK;
-                if (kStream) {
-                    const int nb = (rows + TOKBOX - 1) / TOKBOX;
-                    mbar_expect_tx(full, L::A_BYTES + nb * TOKBOX * BK * 2);
-                    const int f0 = tile * BM;   // output-feature offset within the group
-                    if (MODE == G1_STREAM) {
-                        int z = g, fl = f0;
-                        const CUtensorMap* wm = &maps.w_a;
-                        if (shared) { z = f0 / p.I; fl = f0 - z * p.I; wm = &maps.w_s; }
-                        tma_load_3d(a, wm, full, kx, fl, z);
-                        tma_load_3d(a + TILE_BYTES, wm, full, kx, p.I + fl, z);
-                    } else if (MODE == G2_STREAM) {
-                        if (shared) {
-                            const int z = kx / p.I;
-                            tma_load_3d(a, &maps.w_s, full, kx - z * p.I, f0, z);
-                        } else {
-                            tma_load_3d(a, &maps.w_a, full, kx, f0, g);
-                        }
-                    } else {   // LM_STREAM
-                        tma_load_3d(a, &maps.w_a, full, kx, f0, 0);
+        WorkIter<MODE> it;
+        it.init(p, sched, c, nct);
+        Work w;
+        while (ok && it.next(p, sched, w)) {
+            for (int kt = w.k0; kt < w.k1; ++kt, ++q_issued) {
+                const int stage = q_issued % ST;
+                const uint32_t phase = static_cast<uint32_t>(q_issued / ST) & 1u;
+                const uint32_t a = sbase + stage * L::STAGE, b = a + L::A_BYTES;
+                const uint32_t full = smem_addr(&bar_full[stage]);
+                if (q_issued >= npre) {
+                    if (!mbar_wait(smem_addr(&bar_empty[stage]), phase ^ 1u, lim, &abort_sh)) {
+                        ok = false;
+                        break;
                     }
-                    const CUtensorMap* tm = shared ? &maps.tok_s : &maps.tok_r;
-                    for (int j = 0; j < nb; ++j)
-                        tma_load_3d(b + j * TOKBOX * BK * 2, tm, full, kx, row0 + j * TOKBOX, 0);
-                } else {
-                    mbar_expect_tx(full, L::A_BYTES + (MODE == G1_TILED ? 2 * TILE_BYTES : p.bn * BK * 2));
-                    const CUtensorMap* tm = shared ? &maps.tok_s : &maps.tok_r;
-                    tma_load_3d(a, tm, full, kx, row0 + m0, 0);
-                    if (MODE == G1_TILED) {
-                        const int f0 = tile * BM;
-                        int z = g, fl = f0;
-                        const CUtensorMap* wm = &maps.w_a;
-                        if (shared) { z = f0 / p.I; fl = f0 - z * p.I; wm = &maps.w_s; }
-                        tma_load_3d(b, wm, full, kx, fl, z);
-                        tma_load_3d(b + TILE_BYTES, wm, full, kx, p.I + fl, z);
-                    } else {
-                        const int n0 = tile * p.bn;
-                        for (int j = 0; j < p.bn / BM; ++j) {
-                            if (shared) {
-                                const int z = kx / p.I;
-                                tma_load_3d(b + j * TILE_BYTES, &maps.w_s, full, kx - z * p.I, n0 + j * BM, z);
-                            } else {
-                                tma_load_3d(b + j * TILE_BYTES, &maps.w_a, full, kx, n0 + j * BM, g);
-                            }
-                        }
-                    }
+                    mbar_expect_tx_only(full, weight_bytes());
+                    weight_loads(w, kt, a, b, full);
                 }
-            }
-            issued |= 1u << stage;
-            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-            if (++stage == ST) { stage = 0; phase ^= 1u; }
-            return true;
-        };
-        if (kStream) {
-            for (int pos = rb; pos < re && ok;) {
-                const Seg sg = stream_seg<MODE>(p, sched, pos, re);
-                for (int kt = sg.k0; kt < sg.k1 && ok; ++kt)
-                    ok = produce_kstep(sg.g, sg.tile, kt, sched.rows[sg.g], sched.row0[sg.g], 0);
-                pos += sg.k1 - sg.k0;
-            }
-        } else {
-            for (int t = c; t < total && ok; t += nct) {
-                const int g = find_group(sched, t);
-                const int local = t - sched.prefix[g];
-                const int nt = group_ntiles<MODE>(p, g);
-                const int m = local / nt, n = local - m * nt;
-                const int kt_n = group_ktiles<MODE>(p, g);
-                for (int kt = 0; kt < kt_n && ok; ++kt)
-                    ok = produce_kstep(g, n, kt, sched.rows[g], sched.row0[g], m * BM);
+                token_loads(w, kt, a, b, full);   // arrives on `full` with the token bytes
             }
         }
         if (!ok) {
             report_status(p.status, MS_ERR_TIMEOUT);
             abort_sh = 1;
         }
-        // drain: every load this thread issued must land before the CTA exits
-        for (int s2 = 0; s2 < ST; ++s2)
-            if ((issued >> s2) & 1u) {
-                volatile int never = 0;
-                if (!mbar_wait(smem_addr(&bar_full[s2]), (issued_par >> s2) & 1u, lim, &never))
-                    report_status(p.status, MS_ERR_TIMEOUT);
-            }
+        // drain: every load this thread issued lands before the CTA exits.  A
+        // step whose weight half was prefetched but whose token half was never
+        // issued (only possible if the loop stopped early) gets its arrival so
+        // that its phase can complete once the weights land.
+        for (int q = q_issued; q < npre; ++q) mbar_arrive(smem_addr(&bar_full[q]));
+        const int q_end = q_issued > npre ? q_issued : npre;
+        for (int s2 = 0; s2 < ST && s2 < q_end; ++s2) {
+            const int q_last = s2 + ((q_end - 1 - s2) / ST) * ST;
+            volatile int never = 0;
+            if (!mbar_wait(smem_addr(&bar_full[s2]), static_cast<uint32_t>(q_last / ST) & 1u, lim, &never))
+                report_status(p.status, MS_ERR_TIMEOUT);
+        }
+        tstamp(p, MODE, TS_PRODUCER_DONE);
       }
       __syncwarp();   // lanes 1..31 wait here so the warp reaches the final barrier converged
     } else if (warp == 1) {
       if (lane == 0) {
         // ---------------------------------------------------- MMA issuer (one thread)
-        int stage = 0;
-        uint32_t phase = 0;
-        int acc = 0;
+        int q = 0, acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
-        auto mma_tile = [&](int rows, int k0, int k1) -> bool {
-            if (!mbar_wait(smem_addr(&bar_tempty[acc]), acc_phase ^ 1u, lim, &abort_sh)) return false;
+        WorkIter<MODE> it;
+        it.init(p, sched, c, nct);
+        Work w;
+        while (ok && it.next(p, sched, w)) {
+            if (!mbar_wait(smem_addr(&bar_tempty[acc]), acc_phase ^ 1u, lim, &abort_sh)) { ok = false; break; }
             tc_fence_after();
             uint32_t n_mma;
-            if (kStream) {
-                n_mma = static_cast<uint32_t>((rows + 15) / 16 * 16);
-            } else {
-                n_mma = MODE == G1_TILED ? 256u : static_cast<uint32_t>(p.bn);
-            }
+            if (kStream) n_mma = static_cast<uint32_t>((sched.rows[w.g] + 15) / 16 * 16);
+            else n_mma = MODE == G1_TILED ? 256u : static_cast<uint32_t>(p.bn);
             const uint32_t idesc = idesc_bf16_f32(BM, n_mma);
             const uint32_t d0 = tmem_base + acc * 256;
-            for (int kt = k0; kt < k1; ++kt) {
-                if (!mbar_wait(smem_addr(&bar_full[stage]), phase, lim, &abort_sh)) return false;
-                tc_fence_after();
-                {
-                    const uint32_t a = sbase + stage * L::STAGE;
-                    const uint32_t b = a + L::A_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint32_t accum = (kt > k0 || kk > 0) ? 1u : 0u;
-                        const uint64_t bd = smem_desc_sw128(b + kk * 32);
-                        mma_bf16(d0, smem_desc_sw128(a + kk * 32), bd, idesc, accum);
-                        if (MODE == G1_STREAM)
-                            mma_bf16(d0 + 128, smem_desc_sw128(a + TILE_BYTES + kk * 32), bd, idesc, accum);
-                    }
-                    mma_commit(smem_addr(&bar_empty[stage]));
+            for (int kt = w.k0; kt < w.k1; ++kt, ++q) {
+                const int stage = q % ST;
+                if (!mbar_wait(smem_addr(&bar_full[stage]), static_cast<uint32_t>(q / ST) & 1u, lim, &abort_sh)) {
+                    ok = false;
+                    break;
                 }
-                if (++stage == ST) { stage = 0; phase ^= 1u; }
+                if (q == 0) tstamp(p, MODE, TS_FIRST_DATA);
+                tc_fence_after();
+                const uint32_t a = sbase + stage * L::STAGE;
+                const uint32_t b = a + L::A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint32_t accum = (kt > w.k0 || kk > 0) ? 1u : 0u;
+                    const uint64_t bd = smem_desc_sw128(b + kk * 32);
+                    mma_bf16(d0, smem_desc_sw128(a + kk * 32), bd, idesc, accum);
+                    if (MODE == G1_STREAM)
+                        mma_bf16(d0 + 128, smem_desc_sw128(a + TILE_BYTES + kk * 32), bd, idesc, accum);
+                }
+                mma_commit(smem_addr(&bar_empty[stage]));
             }
+            if (!ok) break;
             mma_commit(smem_addr(&bar_tfull[acc]));
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
-            return true;
-        };
-        if (kStream) {
-            for (int pos = rb; pos < re && ok;) {
-                const Seg sg = stream_seg<MODE>(p, sched, pos, re);
-                ok = mma_tile(sched.rows[sg.g], sg.k0, sg.k1);
-                pos += sg.k1 - sg.k0;
-            }
-        } else {
-            for (int t = c; t < total && ok; t += nct) {
-                const int g = find_group(sched, t);
-                ok = mma_tile(sched.rows[g], 0, group_ktiles<MODE>(p, g));
-            }
         }
         if (!ok) {
             report_status(p.status, MS_ERR_TIMEOUT);
             abort_sh = 1;
         }
+        tstamp(p, MODE, TS_LAST_MMA);
         // drain: all MMAs issued by this thread complete before TMEM is freed
         mma_commit(smem_addr(&bar_drain));
         volatile int never = 0;
@@ -454,35 +554,56 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
     } else {
         // ---------------------------------------------------- epilogue (4 warps)
-        const int q = warp & 3;               // TMEM lane quadrant of this warp
-        const int r_in = q * 32 + lane;       // accumulator row held by this thread
+        const int q4 = warp & 3;              // TMEM lane quadrant of this warp
+        const int r_in = q4 * 32 + lane;      // accumulator row held by this thread
         const int etid = threadIdx.x - 64;    // 0..127
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
         const int ldh_r = p.I, ldh_s = p.S * p.I;
+        const int total = sched.prefix[sched.ngroups];
         auto tmem_at = [&](int col) -> uint32_t {
-            return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256 + col);
+            return tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) + static_cast<uint32_t>(acc * 256 + col);
         };
-        if (kStream) {
-            const int slot_floats = BM * NMAX * (kG1 ? 2 : 1);
-            for (int pos = rb; pos < re && ok;) {
-                const Seg sg = stream_seg<MODE>(p, sched, pos, re);
-                pos += sg.k1 - sg.k0;
-                if (!epi_wait(smem_addr(&bar_tfull[acc]), acc_phase, lim, &abort_sh, etid, go_sh[acc])) {
-                    ok = false;
-                    break;
+        // one finished output value of the streaming schedule (row r_in of the tile, token t)
+        auto store_stream = [&](bool shared, int row0, int f, int t, float va, float vb) {
+            if (MODE == G1_STREAM) {
+                __nv_bfloat16* dst = shared ? p.h_sh + static_cast<size_t>(t) * ldh_s + f
+                                            : p.h_perm + static_cast<size_t>(row0 + t) * ldh_r + f;
+                *dst = __float2bfloat16_rn(silu_mul(va, vb));
+            } else if (MODE == G2_STREAM) {
+                if (shared) {
+                    p.y_sh[static_cast<size_t>(t) * p.H + f] = va;
+                } else if (p.y_bf16) {
+                    reinterpret_cast<__nv_bfloat16*>(p.y_perm)[static_cast<size_t>(row0 + t) * p.H + f] =
+                        __float2bfloat16_rn(va);
+                } else {
+                    reinterpret_cast<float*>(p.y_perm)[static_cast<size_t>(row0 + t) * p.H + f] = va;
                 }
-                tc_fence_after();
-                const int g = sg.g;
-                const bool shared = p.offsets != nullptr && g == p.E;
-                const int rows = sched.rows[g], row0 = sched.row0[g];
-                const int f = sg.tile * BM + r_in;       // output feature of this thread
+            } else {
+                p.logits[static_cast<size_t>(t) * p.V + f] = __float2bfloat16_rn(va);
+            }
+        };
+        WorkIter<MODE> it;
+        it.init(p, sched, c, nct);
+        Work w;
+        while (ok && it.next(p, sched, w)) {
+            if (!epi_wait(smem_addr(&bar_tfull[acc]), acc_phase, lim, &abort_sh, etid, go_sh[acc])) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int g = w.g;
+            const bool shared = p.offsets != nullptr && g == p.E;
+            const int rows = sched.rows[g], row0 = sched.row0[g];
+            if (kStream) {
+                const int slot_floats = BM * NMAX * (kG1 ? 2 : 1);
+                const int f = w.n * BM + r_in;          // output feature of this thread
                 const int nch = (rows + 15) / 16;
-                const bool whole = sg.k0 == 0 && sg.k1 == sg.kt;
+                const bool whole = w.k0 == 0 && w.k1 == w.kt;
                 float* my_slot = nullptr;
                 if (!whole) {
-                    const bool first = range_begin(c, total, nct) >= sg.tile_start;
+                    const bool first = range_begin(c, total, nct) >= w.tile_start;
                     my_slot = p.partials + static_cast<size_t>(2 * c + (first ? 0 : 1)) * slot_floats;
                 }
                 for (int ch = 0; ch < nch; ++ch) {
@@ -501,24 +622,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int t = ch * 16 + j;
-                        if (t >= rows) break;
-                        if (MODE == G1_STREAM) {
-                            const float h = silu_mul(va[j], vb[j]);
-                            __nv_bfloat16* dst = shared ? p.h_sh + static_cast<size_t>(t) * ldh_s + f
-                                                        : p.h_perm + static_cast<size_t>(row0 + t) * ldh_r + f;
-                            *dst = __float2bfloat16_rn(h);
-                        } else if (MODE == G2_STREAM) {
-                            if (shared) {
-                                p.y_sh[static_cast<size_t>(t) * p.H + f] = va[j];
-                            } else if (p.y_bf16) {
-                                reinterpret_cast<__nv_bfloat16*>(p.y_perm)[static_cast<size_t>(row0 + t) * p.H + f] =
-                                    __float2bfloat16_rn(va[j]);
-                            } else {
-                                reinterpret_cast<float*>(p.y_perm)[static_cast<size_t>(row0 + t) * p.H + f] = va[j];
-                            }
-                        } else {
-                            p.logits[static_cast<size_t>(t) * p.V + f] = __float2bfloat16_rn(va[j]);
-                        }
+                        if (t < rows) store_stream(shared, row0, f, t, va[j], kG1 ? vb[j] : 0.f);
                     }
                 }
                 tc_fence_before();
@@ -528,12 +632,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (acc == 0) acc_phase ^= 1u;
                 if (whole) continue;
                 // ---- split tile: the last contributor sums the partials in CTA order
-                const int c_first = cta_of(sg.tile_start, total, nct);
-                const int c_last = cta_of(sg.tile_start + sg.kt - 1, total, nct);
+                const int c_first = cta_of(w.tile_start, total, nct);
+                const int c_last = cta_of(w.tile_start + w.kt - 1, total, nct);
                 int nparts = 0;
                 for (int c2 = c_first; c2 <= c_last; ++c2)
                     if (range_begin(c2 + 1, total, nct) > range_begin(c2, total, nct)) ++nparts;
-                int32_t* ctr = p.counters + static_cast<size_t>(g) * p.max_tiles + sg.tile;
+                int32_t* ctr = p.counters + static_cast<size_t>(g) * p.max_tiles + w.n;
                 __threadfence();
                 epi_bar();
                 if (etid == 0) {
@@ -552,7 +656,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const long b2 = range_begin(c2, total, nct);
                         if (range_begin(c2 + 1, total, nct) <= b2) continue;
                         const float* sl = p.partials +
-                                          static_cast<size_t>(2 * c2 + (b2 < sg.tile_start ? 1 : 0)) * slot_floats;
+                                          static_cast<size_t>(2 * c2 + (b2 < w.tile_start ? 1 : 0)) * slot_floats;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             va[j] += __ldcg(sl + (ch * 16 + j) * BM + r_in);
@@ -562,44 +666,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int t = ch * 16 + j;
-                        if (t >= rows) break;
-                        if (MODE == G1_STREAM) {
-                            const float h = silu_mul(va[j], vb[j]);
-                            __nv_bfloat16* dst = shared ? p.h_sh + static_cast<size_t>(t) * ldh_s + f
-                                                        : p.h_perm + static_cast<size_t>(row0 + t) * ldh_r + f;
-                            *dst = __float2bfloat16_rn(h);
-                        } else if (MODE == G2_STREAM) {
-                            if (shared) {
-                                p.y_sh[static_cast<size_t>(t) * p.H + f] = va[j];
-                            } else if (p.y_bf16) {
-                                reinterpret_cast<__nv_bfloat16*>(p.y_perm)[static_cast<size_t>(row0 + t) * p.H + f] =
-                                    __float2bfloat16_rn(va[j]);
-                            } else {
-                                reinterpret_cast<float*>(p.y_perm)[static_cast<size_t>(row0 + t) * p.H + f] = va[j];
-                            }
-                        } else {
-                            p.logits[static_cast<size_t>(t) * p.V + f] = __float2bfloat16_rn(va[j]);
-                        }
+                        if (t < rows) store_stream(shared, row0, f, t, va[j], kG1 ? vb[j] : 0.f);
                     }
                 }
-            }
-        } else {
-            for (int t = c; t < total && ok; t += nct) {
-                if (!epi_wait(smem_addr(&bar_tfull[acc]), acc_phase, lim, &abort_sh, etid, go_sh[acc])) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const int g = find_group(sched, t);
-                const bool shared = p.offsets != nullptr && g == p.E;
-                const int local = t - sched.prefix[g];
-                const int nt = group_ntiles<MODE>(p, g);
-                const int m = local / nt, n = local - m * nt;
-                const int rr = m * BM + r_in;                 // row within the group
-                const bool valid = rr < sched.rows[g];
-                const size_t orow = static_cast<size_t>(shared ? rr : sched.row0[g] + rr);
+            } else {
+                const int rr = w.m0 + r_in;                  // row within the group
+                const bool valid = rr < rows;
+                const size_t orow = static_cast<size_t>(shared ? rr : row0 + rr);
                 if (MODE == G1_TILED) {
-                    const int f0 = n * BM;
+                    const int f0 = w.n * BM;
                     __nv_bfloat16* dst = shared ? p.h_sh + orow * ldh_s + f0 : p.h_perm + orow * ldh_r + f0;
                     for (int ch = 0; ch < BM / 16; ++ch) {
                         float g16[16], u16[16];
@@ -618,7 +693,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         }
                     }
                 } else {
-                    const int n0 = n * p.bn;
+                    const int n0 = w.n * p.bn;
                     for (int ch = 0; ch < p.bn / 16; ++ch) {
                         float v16[16];
                         tmem_ld16(tmem_at(ch * 16), v16);
@@ -653,11 +728,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (etid == 0) report_status(p.status, MS_ERR_TIMEOUT);
             abort_sh = 1;
         }
+        if (etid == 0) tstamp(p, MODE, TS_EPI_DONE);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+    if (threadIdx.x == 32) tstamp(p, MODE, TS_EXIT);
 }
 
 // ------------------------------------------------------------ prep kernel
@@ -730,6 +807,13 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1,
     return r == CUDA_SUCCESS;
 }
 
+// Packed weight tensor [n][rows/128][cols/64][128][64] viewed as rank 3:
+// 64-element rows, rows*cols/64 of them per matrix, n matrices.  One box of
+// 64 x 128 is one contiguous 16 KB tile.
+static bool make_packed_map(CUtensorMap* m, const void* base, int rows, int cols, int n) {
+    return make_map(m, base, BK, static_cast<uint64_t>(rows) * cols / BK, n, BM);
+}
+
 template <int MODE, int NMAX>
 static ms_status launch_gemm(int id, const Maps& maps, const Params& prm, cudaStream_t s) {
     using L = Layout<MODE, NMAX>;
@@ -755,6 +839,9 @@ static ms_status launch_stream(int id, int nmax, const Maps& maps, const Params&
         default: return launch_gemm<MODE, 128>(id, maps, prm, s);
     }
 }
+
+static uint64_t* g_dtrace = nullptr;
+void set_device_trace(void* buf) { g_dtrace = static_cast<uint64_t*>(buf); }
 
 static int stream_nmax(int T) {
     int n = 16;
@@ -836,16 +923,17 @@ ms_status ffn_launch(const void* x, const int32_t* offsets, const int32_t* perm,
     prm.status = w.status;
     prm.max_tiles = w.max_tiles;
     prm.wait_limit_ns = wait_limit_ns();
+    prm.dtrace = g_dtrace;
     const int ngroups = E + (S > 0 ? 1 : 0);
     const uint32_t tok_box = stream ? TOKBOX : BM;
     const void* x_tok_s = stream ? static_cast<const void*>(w.x_pad) : x;
     const int x_rows = stream ? w.t_pad : T;
     // 2. GEMM1: gate/up + SwiGLU -> h
     Maps m1{};
-    bool ok = make_map(&m1.w_a, wgu, H, 2 * I, E, BM) &&
+    bool ok = make_packed_map(&m1.w_a, wgu, 2 * I, H, E) &&
               make_map(&m1.tok_r, w.x_perm, H, w.rows_pad, 1, tok_box) &&
               make_map(&m1.tok_s, x_tok_s, H, x_rows, 1, tok_box);
-    ok = ok && (S > 0 ? make_map(&m1.w_s, wsgu, H, 2 * I, S, BM) : make_map(&m1.w_s, wgu, H, 2 * I, E, BM));
+    ok = ok && (S > 0 ? make_packed_map(&m1.w_s, wsgu, 2 * I, H, S) : make_packed_map(&m1.w_s, wgu, 2 * I, H, E));
     if (!ok) return MS_ERR_CUDA;
     prm.counters = w.counters;
     ms_status st = stream ? launch_stream<G1_STREAM>(K_GEMM1_STREAM, stream_nmax(T), m1, prm, s)
@@ -854,9 +942,9 @@ ms_status ffn_launch(const void* x, const int32_t* offsets, const int32_t* perm,
     // 3. GEMM2: down projection -> y_perm, y_shared
     Maps m2{};
     const int hs_cols = S > 0 ? S * I : BK;
-    ok = make_map(&m2.w_a, wd, I, H, E, BM) && make_map(&m2.tok_r, w.h_perm, I, w.rows_pad, 1, tok_box) &&
+    ok = make_packed_map(&m2.w_a, wd, H, I, E) && make_map(&m2.tok_r, w.h_perm, I, w.rows_pad, 1, tok_box) &&
          make_map(&m2.tok_s, w.h_sh, hs_cols, w.t_pad, 1, tok_box);
-    ok = ok && (S > 0 ? make_map(&m2.w_s, wsd, I, H, S, BM) : make_map(&m2.w_s, wd, I, H, E, BM));
+    ok = ok && (S > 0 ? make_packed_map(&m2.w_s, wsd, H, I, S) : make_packed_map(&m2.w_s, wd, H, I, E));
     if (!ok) return MS_ERR_CUDA;
     prm.counters = w.counters + ngroups * w.max_tiles;
     return stream ? launch_stream<G2_STREAM>(K_GEMM2_STREAM, stream_nmax(T), m2, prm, s)
@@ -902,7 +990,7 @@ ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* l
                               static_cast<__nv_bfloat16*>(nullptr), w.x_pad, BM, w.counters, V / BM, w.status);
         if (st != MS_OK) return st;
         Maps m{};
-        bool ok = make_map(&m.w_a, wlm, H, V, 1, BM) && make_map(&m.w_s, wlm, H, V, 1, BM) &&
+        bool ok = make_packed_map(&m.w_a, wlm, V, H, 1) && make_packed_map(&m.w_s, wlm, V, H, 1) &&
                   make_map(&m.tok_r, w.x_pad, H, BM, 1, TOKBOX) && make_map(&m.tok_s, w.x_pad, H, BM, 1, TOKBOX);
         if (!ok) return MS_ERR_CUDA;
         Params prm{};
@@ -915,6 +1003,7 @@ ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* l
         prm.status = w.status;
         prm.max_tiles = V / BM;
         prm.wait_limit_ns = wait_limit_ns();
+        prm.dtrace = g_dtrace;
         st = launch_stream<LM_STREAM>(K_LM_HEAD, stream_nmax(tc), m, prm, s);
         if (st != MS_OK) return st;
     }

@@ -16,6 +16,7 @@ enum KernelId : int {
     K_RMSNORM = 0,
     K_ROUTE_ROWS,
     K_ROUTE_TILED,
+    K_ROUTE_CLUSTER,
     K_PERMUTE_COUNT,
     K_PERMUTE_SCATTER,
     K_FFN_PREP,
@@ -27,7 +28,9 @@ enum KernelId : int {
     K_COMBINE,
     K_VERIFY_PARTIAL,
     K_VERIFY_FINAL,
+    K_VERIFY_CLUSTER,
     K_WAIT_PROBE,
+    K_PACK,
     K_COUNT
 };
 const char* kernel_name(int id);
@@ -53,6 +56,34 @@ inline ms_status launch(int id, void (*kernel)(KArgs...), dim3 grid, dim3 block,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    trace_mark(id, s, false);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    trace_mark(id, s, true);
+    if (e != cudaSuccess) {
+        set_cuda_error(e);
+        return MS_ERR_CUDA;
+    }
+    return MS_OK;
+}
+
+// Same, launched as thread-block clusters of `cluster_x` CTAs along x.
+template <typename... KArgs, typename... Args>
+inline ms_status launch_cluster(int id, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                cudaStream_t s, int cluster_x, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     trace_mark(id, s, false);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
     trace_mark(id, s, true);
@@ -120,6 +151,31 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+
+// ---- thread-block clusters: distributed shared memory and the cluster barrier
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Store v into the same shared-memory variable of CTA `rank` of this cluster.
+__device__ __forceinline__ void st_cluster_f32(const void* local, uint32_t rank, float v) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(local));
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_s32(const void* local, uint32_t rank, int v) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(local));
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
+}
+// Every thread of every CTA of the cluster must reach this; it orders the
+// stores above before the loads after it, cluster-wide.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {

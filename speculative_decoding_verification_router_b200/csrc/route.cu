@@ -181,10 +181,118 @@ __global__ void __launch_bounds__(256) route_tiled_kernel(const __nv_bfloat16* _
     }
 }
 
+// Small T: one cluster of RC_CTAS CTAs per token.  CTA r computes the logits
+// of experts [r*E/RC_CTAS, (r+1)*E/RC_CTAS) -- one warp per expert, float4
+// loads of W_r spread over RC_CTAS SMs -- and stores them into CTA 0's shared
+// memory (distributed shared memory); after the cluster barrier CTA 0 runs the
+// softmax and top-k.  With NORM the CTAs first RMS-normalise the fp32 residual
+// row themselves (eps, unit gain) and CTA 0 writes the bf16 result, so the
+// layer needs no separate normalisation kernel.
+constexpr int RC_CTAS = 8;
+
+template <bool NORM>
+__global__ void __launch_bounds__(256) route_cluster_kernel(const void* __restrict__ xin,
+                                                            const float* __restrict__ wr,
+                                                            const float* __restrict__ bias, int T, int H,
+                                                            int E, int k, int renorm, float eps,
+                                                            int32_t* __restrict__ idx, float* __restrict__ w,
+                                                            __nv_bfloat16* __restrict__ xhat_out) {
+    extern __shared__ float smem[];
+    float* xs = smem;        // [H] the token's normalised activation (bf16 values)
+    float* z = smem + H;     // [E] logits, filled by every CTA of the cluster
+    __shared__ float red[8];
+    grid_dep_wait();
+    grid_dep_launch();
+    const uint32_t rank = cluster_rank();
+    const int t = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (NORM) {
+        const float4* row = reinterpret_cast<const float4*>(static_cast<const float*>(xin) + static_cast<size_t>(t) * H);
+        float ss = 0.f;
+        for (int i = threadIdx.x; i < H / 4; i += blockDim.x) {
+            const float4 v = __ldg(row + i);
+            ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) red[warp] = ss;
+        __syncthreads();
+        float tot = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tot += red[i];
+        const float inv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+        for (int i = threadIdx.x; i < H / 4; i += blockDim.x) {
+            const float4 v = __ldg(row + i);
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x * inv, v.y * inv);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z * inv, v.w * inv);
+            xs[4 * i] = __low2float(lo);
+            xs[4 * i + 1] = __high2float(lo);
+            xs[4 * i + 2] = __low2float(hi);
+            xs[4 * i + 3] = __high2float(hi);
+            if (rank == 0) {
+                __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(xhat_out + static_cast<size_t>(t) * H);
+                o[2 * i] = lo;
+                o[2 * i + 1] = hi;
+            }
+        }
+    } else {
+        const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(xin) + static_cast<size_t>(t) * H);
+        for (int i = threadIdx.x; i < H / 8; i += blockDim.x) {
+            const uint4 u = __ldg(xr + i);
+            const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                xs[8 * i + 2 * j] = __uint_as_float(q[j] << 16);
+                xs[8 * i + 2 * j + 1] = __uint_as_float(q[j] & 0xffff0000u);
+            }
+        }
+    }
+    __syncthreads();
+    const int per = (E + RC_CTAS - 1) / RC_CTAS;
+    const int e0 = static_cast<int>(rank) * per;
+    const int e1 = e0 + per < E ? e0 + per : E;
+    for (int e = e0 + warp; e < e1; e += 8) {
+        const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * H);
+        float acc = 0.f;
+#pragma unroll 4
+        for (int h4 = lane; h4 < H / 4; h4 += 32) {
+            const float4 a = __ldg(wrow + h4);
+            const float4 b = *reinterpret_cast<const float4*>(xs + 4 * h4);
+            acc = fmaf(a.x, b.x, acc);
+            acc = fmaf(a.y, b.y, acc);
+            acc = fmaf(a.z, b.z, acc);
+            acc = fmaf(a.w, b.w, acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) st_cluster_f32(&z[e], 0, bias ? acc + __ldg(bias + static_cast<size_t>(t) * E + e) : acc);
+    }
+    cluster_sync_all();
+    if (rank == 0 && warp == 0)
+        warp_topk_softmax(z, E, k, renorm, idx + static_cast<size_t>(t) * k, w + static_cast<size_t>(t) * k, lane);
+}
+
+ms_status route_cluster_launch(const void* xin, bool norm, float eps, const float* wr, const float* bias, int T,
+                               int H, int E, int k, int renorm, int32_t* idx, float* w, void* xhat_out,
+                               cudaStream_t s) {
+    const size_t smem = sizeof(float) * static_cast<size_t>(H + E);
+    static bool set = false;
+    if (!set) {
+        cudaFuncSetAttribute(route_cluster_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaFuncSetAttribute(route_cluster_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        set = true;
+    }
+    auto* xo = reinterpret_cast<__nv_bfloat16*>(xhat_out);
+    if (norm)
+        return launch_cluster(K_ROUTE_CLUSTER, route_cluster_kernel<true>, dim3(RC_CTAS, T), dim3(256), smem, s,
+                              RC_CTAS, xin, wr, bias, T, H, E, k, renorm, eps, idx, w, xo);
+    return launch_cluster(K_ROUTE_CLUSTER, route_cluster_kernel<false>, dim3(RC_CTAS, T), dim3(256), smem, s,
+                          RC_CTAS, xin, wr, bias, T, H, E, k, renorm, eps, idx, w, xo);
+}
+
 ms_status route_launch(const void* x, const float* wr, const float* bias, int T, int H, int E,
                        int k, int renorm, int32_t* idx, float* w, cudaStream_t s) {
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-    if (T >= 1024 && E <= RT_EXP && H % RT_K == 0) {
+    if (T < 1024) return route_cluster_launch(x, false, 0.f, wr, bias, T, H, E, k, renorm, idx, w, nullptr, s);
+    if (E <= RT_EXP && H % RT_K == 0) {
         dim3 grid((T + RT_TOK - 1) / RT_TOK);
         return launch(K_ROUTE_TILED, route_tiled_kernel, grid, dim3(256), 0, s, xb, wr, bias, T, H,
                       E, k, renorm, idx, w);

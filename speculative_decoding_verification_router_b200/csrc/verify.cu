@@ -123,6 +123,159 @@ __global__ void __launch_bounds__(128) verify_final_kernel(const float* __restri
     }
 }
 
+// Single-kernel verification: one thread-block cluster per sequence, CTA r of
+// the cluster scans chunk r % P of row r / P with 16-byte loads (several in
+// flight per thread), reduces (max, lowest index) in the block and stores the
+// result into CTA 0's shared memory; after the cluster barrier one warp of
+// CTA 0 merges the P chunks of each row and runs the prefix match.
+constexpr int VC_THREADS = 512;
+constexpr int VC_MAX = 16;
+constexpr int VC_UNROLL = 4;
+
+template <typename TL>
+__global__ void __launch_bounds__(VC_THREADS) verify_cluster_kernel(const TL* __restrict__ logits, int K, int V,
+                                                                    int P, int chunk, int vec_ok,
+                                                                    const int32_t* __restrict__ draft,
+                                                                    int32_t* __restrict__ argmax,
+                                                                    int32_t* __restrict__ committed,
+                                                                    int32_t* __restrict__ n_committed) {
+    constexpr int VEC = 16 / sizeof(TL);
+    __shared__ float cv[VC_MAX];
+    __shared__ int ci[VC_MAX];
+    __shared__ float sv[VC_THREADS / 32];
+    __shared__ int si[VC_THREADS / 32];
+    grid_dep_wait();
+    grid_dep_launch();
+    const uint32_t rank = cluster_rank();
+    const int b = blockIdx.y;
+    const int j = static_cast<int>(rank) / P, pc = static_cast<int>(rank) % P;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    if (j <= K) {
+        const int begin = pc * chunk;
+        const int end = min(V, begin + chunk);
+        const TL* row = logits + (static_cast<size_t>(b) * (K + 1) + j) * V;
+        int tail_begin = begin;
+        if (vec_ok && end > begin) {
+            const int nvec = (end - begin) / VEC;
+            for (int q0 = threadIdx.x; q0 < nvec; q0 += VC_UNROLL * VC_THREADS) {
+                float v[VC_UNROLL][VEC];
+#pragma unroll
+                for (int u = 0; u < VC_UNROLL; ++u) {
+                    const int q = q0 + u * VC_THREADS;
+                    if (q < nvec) vec_load(row + begin + q * VEC, v[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < VC_UNROLL; ++u) {
+                    const int q = q0 + u * VC_THREADS;
+                    if (q < nvec) {
+#pragma unroll
+                        for (int e = 0; e < VEC; ++e) argmax_merge(bv, bi, v[u][e], begin + q * VEC + e);
+                    }
+                }
+            }
+            tail_begin = begin + nvec * VEC;
+        }
+        for (int i = tail_begin + threadIdx.x; i < end; i += VC_THREADS)
+            argmax_merge(bv, bi, scalar_load(row + i), i);
+    }
+    warp_argmax(bv, bi);
+    if (lane == 0) {
+        sv[warp] = bv;
+        si[warp] = bi;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        bv = lane < VC_THREADS / 32 ? sv[lane] : -INFINITY;
+        bi = lane < VC_THREADS / 32 ? si[lane] : 0x7fffffff;
+        warp_argmax(bv, bi);
+        if (lane == 0) {
+            st_cluster_f32(&cv[rank], 0, bv);
+            st_cluster_s32(&ci[rank], 0, bi);
+        }
+    }
+    cluster_sync_all();
+    if (rank == 0 && warp == 0) {
+        // lane l < (K+1)*P holds chunk l; row r = chunks [r*P, r*P + P)
+        const int n = (K + 1) * P;
+        const float lv = lane < n ? cv[lane] : -INFINITY;
+        const int li = lane < n ? ci[lane] : 0x7fffffff;
+        const int dr = lane < K ? __ldg(draft + static_cast<size_t>(b) * K + lane) : -1;
+        int g[kMaxK + 1];
+#pragma unroll
+        for (int r = 0; r <= kMaxK; ++r) {
+            float mv = (lane >= r * P && lane < r * P + P) ? lv : -INFINITY;
+            int mi = (lane >= r * P && lane < r * P + P) ? li : 0x7fffffff;
+            warp_argmax(mv, mi);
+            g[r] = mi;
+        }
+        // first draft position that disagrees with the verifier's pick
+        const unsigned miss = __ballot_sync(0xffffffffu, lane < K && dr != g[lane < kMaxK ? lane : 0]);
+        if (lane == 0) {
+            const int n_acc = miss ? (__ffs(miss) - 1) : K;
+            int32_t* am = argmax + static_cast<size_t>(b) * (K + 1);
+            int32_t* cm = committed + static_cast<size_t>(b) * (K + 1);
+            for (int r = 0; r <= K; ++r) {
+                am[r] = g[r];
+                cm[r] = r <= n_acc ? g[r] : -1;
+            }
+            n_committed[b] = n_acc + 1;
+        }
+    }
+}
+
+static int verify_cluster_size() {
+    // 16-CTA clusters when the device allows them, else the portable 8
+    static int cs = 0;
+    if (cs == 0) {
+        cs = 8;
+        if (cudaFuncSetAttribute(verify_cluster_kernel<__nv_bfloat16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(verify_cluster_kernel<float>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(16, 1);
+            cfg.blockDim = dim3(VC_THREADS);
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = 16;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, verify_cluster_kernel<__nv_bfloat16>, &cfg) == cudaSuccess && n > 0)
+                cs = 16;
+        }
+        cudaGetLastError();
+    }
+    return cs;
+}
+
+static ms_status verify_cluster_launch(const void* logits, ms_dtype dt, const int32_t* draft, int B, int K, int V,
+                                       int32_t* argmax, int32_t* committed, int32_t* ncom, cudaStream_t s) {
+    const int eb = dt == MS_BF16 ? 2 : 4;
+    const int vec = 16 / eb;
+    const int cs_max = verify_cluster_size();
+    int P = cs_max / (K + 1);
+    const int maxP = (V + 1023) / 1024;
+    if (P > maxP) P = maxP;
+    if (P < 1) P = 1;
+    int chunk = (V + P - 1) / P;
+    chunk = (chunk + vec - 1) / vec * vec;
+    P = (V + chunk - 1) / chunk;
+    const int cs = (K + 1) * P;
+    const int vec_ok = (V % vec == 0) && aligned16(logits);
+    if (dt == MS_BF16)
+        return launch_cluster(K_VERIFY_CLUSTER, verify_cluster_kernel<__nv_bfloat16>, dim3(cs, B), dim3(VC_THREADS), 0,
+                              s, cs, reinterpret_cast<const __nv_bfloat16*>(logits), K, V, P, chunk, vec_ok, draft,
+                              argmax, committed, ncom);
+    return launch_cluster(K_VERIFY_CLUSTER, verify_cluster_kernel<float>, dim3(cs, B), dim3(VC_THREADS), 0, s, cs,
+                          reinterpret_cast<const float*>(logits), K, V, P, chunk, vec_ok, draft, argmax, committed,
+                          ncom);
+}
+
 struct VerifyPlan {
     int P, chunk;
 };
@@ -249,6 +402,11 @@ extern "C" ms_status spec_verify_greedy(const void* logits, ms_dtype logits_dtyp
     if (K > ms::kMaxK) return MS_ERR_UNSUPPORTED;
     if (static_cast<long>(B) * (K + 1) * V > (1L << 40)) return MS_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < ms::verify_ws_bytes(B, K, V)) return MS_ERR_WORKSPACE;
+    // one cluster per sequence when its K+1 rows fit a cluster; the
+    // two-kernel path (partials through ws) otherwise
+    if (K + 1 <= ms::verify_cluster_size())
+        return ms::verify_cluster_launch(logits, logits_dtype, draft, B, K, V, argmax, committed, n_committed,
+                                         static_cast<cudaStream_t>(stream));
     return ms::verify_launch(logits, logits_dtype, draft, B, K, V, argmax, committed, n_committed,
                              ws, static_cast<cudaStream_t>(stream));
 }

@@ -62,6 +62,8 @@ def _load():
         "ms_status_string": (ctypes.c_char_p, [I]),
         "ms_last_cuda_error_string": (ctypes.c_char_p, []),
         "ms_version": (I, []),
+        "moe_pack_weights": (I, [P, I, I, I, P, P]),
+        "ms_set_device_trace": (I, [P, Z]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -127,6 +129,19 @@ def _ws(ws: Optional[Workspace], need: int, device) -> Workspace:
 
 
 # ------------------------------------------------------------------ calls
+
+def pack_weights(w: torch.Tensor, stream=None) -> torch.Tensor:
+    """Repack a bf16 weight stack [n, rows, cols] (or [rows, cols]) into the
+    tile-contiguous layout the GEMM entry points read.  Same shape and dtype;
+    only the element order changes."""
+    _dev(w, torch.bfloat16, "w")
+    shape = w.shape
+    w3 = w.view(1, *shape) if w.dim() == 2 else w
+    n, rows, cols = w3.shape
+    out = torch.empty_like(w)
+    _check(_lib.moe_pack_weights(_p(w3), n, rows, cols, _p(out), _stream(stream)), "moe_pack_weights")
+    return out
+
 
 def rmsnorm(a: torch.Tensor, gamma=None, eps: float = 1e-6, out=None, stream=None) -> torch.Tensor:
     _dev(a, torch.float32, "a")
@@ -267,6 +282,14 @@ def get_wait_limit_ns() -> int:
 
 def debug_bounded_wait(flag: torch.Tensor, expect: int, status: torch.Tensor, stream=None):
     _check(_lib.ms_debug_bounded_wait(_p(flag), int(expect), _p(status), _stream(stream)), "ms_debug_bounded_wait")
+
+
+def set_device_trace(buf: Optional[torch.Tensor]):
+    """Point the GEMMs' per-CTA timeline at `buf` (uint64 tensor, >= 5*256*8), or None to stop."""
+    if buf is None:
+        _check(_lib.ms_set_device_trace(None, 0), "ms_set_device_trace")
+    else:
+        _check(_lib.ms_set_device_trace(_p(buf), buf.numel() * buf.element_size()), "ms_set_device_trace")
 
 
 def trace_enable(capacity: int):

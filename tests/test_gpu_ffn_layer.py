@@ -23,8 +23,10 @@ def ms():
 
 
 def _weights_dev(lw):
-    return (dev(lw.w_gate_up), dev(lw.w_down), None if lw.ws_gate_up is None else dev(lw.ws_gate_up),
-            None if lw.ws_down is None else dev(lw.ws_down))
+    """Expert weights on the device in the packed layout the GEMMs read."""
+    from speculative_decoding_verification_router_b200 import moespec as ms
+    pk = lambda a: None if a is None else ms.pack_weights(dev(a))
+    return pk(lw.w_gate_up), pk(lw.w_down), pk(lw.ws_gate_up), pk(lw.ws_down)
 
 
 def _ffn_case(ms, shp, seed, y_dtype=torch.float32):
@@ -154,7 +156,7 @@ def test_lm_head_parity(ms, T, V):
     H = 1280 if V > 2048 else 256
     x = synth.normal_bf16(0, f"lmx{T}", (T, H), 1.0)
     wl = synth.normal_bf16(0, f"lmw{V}", (V, H), 0.02)
-    out = ms.lm_head(dev(x), dev(wl))
+    out = ms.lm_head(dev(x), ms.pack_weights(dev(wl)))
     torch.cuda.synchronize()
     if V <= 2048:
         ref = oracle.lm_head(oracle.widen_bf16(x), wl)
@@ -166,6 +168,14 @@ def test_lm_head_parity(ms, T, V):
         got = host(out)[:, cols]
     # logits are written in bf16: one bf16 rounding of a ~N(0, 0.5) value
     assert_close(got, ref, max_rel=1e-2, mae=2e-3, what="logits")
+
+
+@pytest.mark.parametrize("n,rows,cols", [(3, 256, 128), (1, 128, 64), (2, 1792, 1280), (1, 384, 896)])
+def test_pack_weights_is_the_tile_permutation(ms, n, rows, cols):
+    w = synth.normal_bf16(0, f"pack{n}x{rows}x{cols}", (n, rows, cols), 1.0)
+    got = ms.bf16_to_bits(ms.pack_weights(dev(w))).reshape(-1)
+    ref = w.reshape(n, rows // 128, 128, cols // 64, 64).transpose(0, 1, 3, 2, 4).reshape(-1)
+    np.testing.assert_array_equal(got, ref)
 
 
 def test_bounded_wait_reports_timeout(ms):
@@ -201,6 +211,6 @@ def test_trace_records_kernels(ms):
         ms.trace_disable()
         ms.trace_reset()
     names = [n for n, _ in recs]
-    assert names == ["rmsnorm", "route_rows", "permute_scatter", "ffn_prep", "gemm1_stream", "gemm2_stream",
-                     "combine"]
+    assert names == ["route_cluster", "permute_scatter", "ffn_prep", "gemm1_stream", "gemm2_stream",
+                     "combine"], names
     assert all(t > 0 for _, t in recs)
