@@ -344,12 +344,14 @@ def run_ours(args, rank, world, local):
     wl = shp.name
     alg = routed_work(prob, ms, stream)
     stream_mode = shp.T <= 128
-    g1 = "gemm1_stream" if stream_mode else "gemm1_tiled"
-    g2 = "gemm2_stream" if stream_mode else "gemm2_tiled"
-    dominant = max((g1, g2), key=lambda n: breakdown.get(n, 0.0))
+    if stream_mode:
+        dominant = max(("gemm1_stream", "gemm2_stream"), key=lambda n: breakdown.get(n, 0.0))
+    else:
+        dominant = max(("gemm1_tiled", "gemm2_tiled"), key=lambda n: breakdown.get(n, 0.0))
+    g1 = "gemm1_tiled"
     dur_s = float(np.mean(per_kernel[dominant])) / 1e3
     if stream_mode:
-        nbytes = alg["g1_bytes"] if dominant == g1 else alg["g2_bytes"]
+        nbytes = {"gemm1_stream": alg["g1_bytes"], "gemm2_stream": alg["g2_bytes"]}[dominant]
         achieved = nbytes / dur_s / 1e9
         roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),

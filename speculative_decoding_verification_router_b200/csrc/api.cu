@@ -27,7 +27,7 @@ void set_device_trace(void*);
 
 static const char* kNames[K_COUNT] = {
     "rmsnorm",        "route_rows",      "route_tiled",     "route_cluster", "permute_count", "permute_scatter",
-    "ffn_prep",       "gemm1_stream",    "gemm2_stream",    "gemm1_tiled",   "gemm2_tiled",
+    "ffn_prep",       "gemm1_stream",    "gemm2_stream",    "gemm1_tiled",   "gemm2_tiled",  "ffn_finish",
     "lm_head_stream", "combine",         "verify_partial",  "verify_final",  "verify_cluster", "wait_probe",
     "pack_weights"};
 

@@ -26,6 +26,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <stdlib.h>
 
 #include "ms_sm100.cuh"
 
@@ -40,7 +41,12 @@ constexpr int TOKBOX = 16;               // token rows per TMA box (streaming)
 constexpr int NTHREADS = 192;
 constexpr int MAX_GROUPS = 257;
 constexpr int TMEM_COLS = 512;
-constexpr int SMEM_BUDGET = 210 * 1024;
+#ifndef MS_SMEM_BUDGET_KB
+#define MS_SMEM_BUDGET_KB 140
+#endif
+// Shared memory for pipeline stages.  More stages means more bytes in flight
+// per SM; beyond what saturates HBM they only lengthen the memory queues.
+constexpr int SMEM_BUDGET = MS_SMEM_BUDGET_KB * 1024;
 
 enum Mode : int { G1_STREAM = 0, G2_STREAM = 1, LM_STREAM = 2, G1_TILED = 3, G2_TILED = 4 };
 
@@ -61,10 +67,9 @@ struct Params {
     int y_bf16;
     float* y_sh;                   // [T][H]
     __nv_bfloat16* logits;         // [T][V]
-    float* partials;               // 2 slots per CTA (streaming)
-    int32_t* counters;             // one per tile (streaming)
+    float* partials;               // 2 partial-sum slots per CTA (streaming)
+    int nct;                       // grid size of the streaming GEMM (for the finish kernel)
     int32_t* status;
-    int max_tiles;                 // tiles per group upper bound (counter stride)
     uint64_t wait_limit_ns;
     uint64_t* dtrace;              // optional per-CTA timeline (see ms_set_device_trace)
 };
@@ -96,10 +101,38 @@ struct Layout {
 // ------------------------------------------------------------ schedule
 struct Sched {
     int ngroups;
-    int prefix[MAX_GROUPS + 1];   // units before group g
+    int prefix[MAX_GROUPS + 1];   // units before group g (k-steps when streaming, tiles when tiled)
+    int tprefix[MAX_GROUPS + 1];  // streaming: output tiles before group g
     int rows[MAX_GROUPS];
     int row0[MAX_GROUPS];
 };
+
+// Inclusive-to-exclusive scan of a[1..n] in place (a[0] = 0), by one warp.
+__device__ __forceinline__ void warp_scan_groups(int* a, int n, int lane) {
+    constexpr int kPer = (MAX_GROUPS + 31) / 32;
+    int loc[kPer];
+    int sum = 0;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int g = lane * kPer + q;
+        loc[q] = g < n ? a[g + 1] : 0;
+        sum += loc[q];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int g = lane * kPer + q;
+        run += loc[q];
+        if (g < n) a[g + 1] = run;
+    }
+    if (lane == 0) a[0] = 0;
+}
 
 template <int MODE>
 __device__ __forceinline__ int group_ktiles(const Params& p, int g) {
@@ -120,11 +153,7 @@ __device__ __forceinline__ int group_ntiles(const Params& p, int g) {
 template <int MODE>
 __device__ void build_schedule(const Params& p, Sched& s) {
     const int tid = threadIdx.x;
-    if (p.offsets == nullptr) {
-        s.ngroups = 1;
-    } else {
-        s.ngroups = p.E + (p.S > 0 ? 1 : 0);
-    }
+    s.ngroups = p.offsets == nullptr ? 1 : p.E + (p.S > 0 ? 1 : 0);
     const int ng = s.ngroups;
     for (int g = tid; g < ng; g += NTHREADS) {
         int rows, row0;
@@ -144,43 +173,21 @@ __device__ void build_schedule(const Params& p, Sched& s) {
         }
         s.rows[g] = rows;
         s.row0[g] = row0;
-        int units = 0;
+        int units = 0, tiles = 0;
         if (rows > 0) {
-            if (Cfg<MODE>::kStream)
-                units = group_ntiles<MODE>(p, g) * group_ktiles<MODE>(p, g);
-            else
+            if (Cfg<MODE>::kStream) {
+                tiles = group_ntiles<MODE>(p, g);
+                units = tiles * group_ktiles<MODE>(p, g);
+            } else {
                 units = ((rows + BM - 1) / BM) * group_ntiles<MODE>(p, g);
+            }
         }
         s.prefix[g + 1] = units;   // scanned below
+        s.tprefix[g + 1] = tiles;
     }
     __syncthreads();
-    if (tid < 32) {
-        // inclusive scan over groups: each lane owns a run of groups
-        constexpr int kPer = (MAX_GROUPS + 31) / 32;
-        const int lane = tid;
-        int loc[kPer];
-        int sum = 0;
-#pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            const int g = lane * kPer + q;
-            loc[q] = g < ng ? s.prefix[g + 1] : 0;
-            sum += loc[q];
-        }
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - sum;
-#pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            const int g = lane * kPer + q;
-            run += loc[q];
-            if (g < ng) s.prefix[g + 1] = run;
-        }
-        if (lane == 0) s.prefix[0] = 0;
-    }
+    if (tid < 32) warp_scan_groups(s.prefix, ng, tid);
+    else if (tid < 64) warp_scan_groups(s.tprefix, ng, tid - 32);
     __syncthreads();
 }
 
@@ -227,63 +234,100 @@ __device__ __forceinline__ Seg stream_seg(const Params& p, const Sched& s, int p
 // one TMEM buffer.  All three roles walk the same sequence.
 struct Work {
     int g, n, m0, k0, k1, kt, tile_start;
+    int rot;   // whole tiles: k-steps are visited as (i + rot) % kt, i = 0..kt-1
 };
+
+// The k-step loaded/multiplied at iteration i of work item w.  Whole tiles
+// start at a CTA-dependent offset so that the CTAs streaming their whole tiles
+// at the same time do not all read the same k offset (same DRAM channels) at
+// once; partial tiles keep their natural order.
+__device__ __forceinline__ int kstep_of(const Work& w, int i) { return w.rot ? (i + w.rot) % w.kt : i; }
+
+// largest g with tprefix[g] <= t
+__device__ __forceinline__ int find_group_tile(const Sched& s, int t) {
+    int lo = 0, hi = s.ngroups - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s.tprefix[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
 
 template <int MODE>
 struct WorkIter {
-    // streaming: this CTA's contiguous k-step range [rb, re), visited in the
-    // order [split tile at the end of the range], then [rb, last_start): the
-    // tiles shared with a neighbour CTA come first, so their fix-up overlaps
-    // the streaming of the whole tiles instead of forming the kernel's tail.
-    // tiled: tiles c, c + nct, ...
-    int rb, re, last_start, pos, state, t, total, nct;
+    // Streaming ("data-parallel + stream-K", split part first): with NT output
+    // tiles in group order and nct CTAs, CTA c owns the D = NT / nct whole
+    // tiles [c*D, c*D + D); the k-steps of the remaining NT - nct*D tiles at the
+    // end of the order (the split region) are divided into nct equal ranges.
+    // A CTA walks its split range first and its whole tiles last, so every
+    // tile shared between CTAs is finished (and its fix-up done) early and the
+    // kernel ends on whole tiles, whose epilogue is a plain store.
+    // Tiled: tiles c, c + nct, ... (round robin).
+    int c, nct, state, pos, re, dp_next, dp_end, t, total;
+    int sk_begin, sk_total;   // split region in absolute k-step positions
 
-    __device__ void init(const Params& p, const Sched& s, int c, int nct_) {
+    __device__ void init(const Params& p, const Sched& s, int c_, int nct_) {
+        c = c_;
         nct = nct_;
         total = s.prefix[s.ngroups];
         if (Cfg<MODE>::kStream) {
-            rb = static_cast<int>(range_begin(c, total, nct));
-            re = static_cast<int>(range_begin(c + 1, total, nct));
-            state = 0;
-            if (re > rb) {
-                const int g = find_group(s, re - 1);
-                const int kt = group_ktiles<MODE>(p, g);
-                const int local = re - 1 - s.prefix[g];
-                const int ts = re - 1 - (local % kt);
-                last_start = ts > rb ? ts : rb;
+            const int nt = s.tprefix[s.ngroups];
+            const int D = nt / nct;
+            dp_next = c * D;
+            dp_end = dp_next + D;
+            const int first_split_tile = nct * D;
+            if (first_split_tile < nt) {
+                const int g = find_group_tile(s, first_split_tile);
+                sk_begin = s.prefix[g] + (first_split_tile - s.tprefix[g]) * group_ktiles<MODE>(p, g);
             } else {
-                last_start = rb;
-                state = 2;
+                sk_begin = total;
             }
+            sk_total = total - sk_begin;
+            pos = sk_range_begin(c);
+            re = sk_range_begin(c + 1);
+            state = 0;
         } else {
             t = c;
         }
     }
+    // first k-step of CTA cc's split range, and the CTA whose range holds `abs`
+    __device__ int sk_range_begin(int cc) const {
+        return sk_begin + static_cast<int>(static_cast<long>(cc) * sk_total / nct);
+    }
+    __device__ int sk_cta_of(int abs) const { return cta_of(abs - sk_begin, sk_total, nct); }
 
     __device__ bool next(const Params& p, const Sched& s, Work& w) {
         if (Cfg<MODE>::kStream) {
-            int from, to;
             if (state == 0) {
-                from = last_start;
-                to = re;
+                if (pos < re) {
+                    const Seg sg = stream_seg<MODE>(p, s, pos, re);
+                    pos += sg.k1 - sg.k0;
+                    w.g = sg.g;
+                    w.n = sg.tile;
+                    w.m0 = 0;
+                    w.k0 = sg.k0;
+                    w.k1 = sg.k1;
+                    w.kt = sg.kt;
+                    w.tile_start = sg.tile_start;
+                    w.rot = 0;
+                    return true;
+                }
                 state = 1;
-                pos = rb;
-            } else if (state == 1 && pos < last_start) {
-                from = pos;
-                to = last_start;
-            } else {
-                return false;
             }
-            const Seg sg = stream_seg<MODE>(p, s, from, to);
-            if (state == 1 && from != last_start) pos = from + (sg.k1 - sg.k0);
-            w.g = sg.g;
-            w.n = sg.tile;
-            w.m0 = 0;
-            w.k0 = sg.k0;
-            w.k1 = sg.k1;
-            w.kt = sg.kt;
-            w.tile_start = sg.tile_start;
-            return true;
+            if (dp_next < dp_end) {
+                const int g = find_group_tile(s, dp_next);
+                w.g = g;
+                w.n = dp_next - s.tprefix[g];
+                w.m0 = 0;
+                w.k0 = 0;
+                w.kt = group_ktiles<MODE>(p, g);
+                w.k1 = w.kt;
+                w.tile_start = s.prefix[g] + w.n * w.kt;
+                w.rot = c % w.kt;
+                ++dp_next;
+                return true;
+            }
+            return false;
         } else {
             if (t >= total) return false;
             const int g = find_group(s, t);
@@ -297,6 +341,7 @@ struct WorkIter {
             w.kt = group_ktiles<MODE>(p, g);
             w.k1 = w.kt;
             w.tile_start = -1;
+            w.rot = 0;
             t += nct;
             return true;
         }
@@ -317,6 +362,54 @@ __device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, uint64_t
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+// Partial-sum slot of a split tile: [half][chunk][row][16].  A thread's 16
+// values of one chunk are 64 contiguous bytes (four 16-byte accesses) and a
+// warp's 32 rows 2 KB, so contributors write and the finisher reads with
+// full-width vector accesses.
+template <int NMAX>
+__device__ __forceinline__ size_t slot_off(int half, int ch, int r) {
+    return ((static_cast<size_t>(half) * (NMAX / 16) + ch) * BM + r) * 16;
+}
+__device__ __forceinline__ void slot_store16(float* dst, const float (&v)[16]) {
+    float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+// v += the 16 values of every contributor's slot, contributors in CTA order;
+// loads of up to four contributors are issued before their additions.
+template <int NMAX, typename SlotOf>
+__device__ __forceinline__ void slot_sum16(SlotOf slot_of, int c_first, int c_last, int half, int ch, int r,
+                                           float (&v)[16]) {
+    int c2 = c_first;
+    while (true) {
+        const float* src[4];
+        int nb = 0;
+        for (; c2 <= c_last && nb < 4; ++c2) {
+            const float* sl = slot_of(c2);
+            if (sl) src[nb++] = sl + slot_off<NMAX>(half, ch, r);
+        }
+        if (nb == 0) break;
+        float4 x[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (u < nb) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) x[u][q] = __ldcg(reinterpret_cast<const float4*>(src[u]) + q);
+            }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (u < nb) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    v[4 * q] += x[u][q].x;
+                    v[4 * q + 1] += x[u][q].y;
+                    v[4 * q + 2] += x[u][q].z;
+                    v[4 * q + 3] += x[u][q].w;
+                }
+            }
+    }
+}
+
 // Row of the packed weight tensor (see pack.cu) that starts the 128-row x
 // 64-column tile at (row r0, k-step kb) of a matrix with `kt` k-steps per row.
 __device__ __forceinline__ int packed_row(int r0, int kb, int kt) { return ((r0 / BM) * kt + kb) * BM; }
@@ -335,7 +428,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __shared__ __align__(8) uint64_t bar_full[ST], bar_empty[ST], bar_tfull[2], bar_tempty[2], bar_drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
-    __shared__ int last_sh;
     __shared__ int go_sh[2];
     __shared__ Sched sched;
 
@@ -433,10 +525,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         it.init(p, sched, c, nct);
         Work w;
         while (npre < ST && it.next(p, sched, w)) {
-            for (int kt = w.k0; kt < w.k1 && npre < ST; ++kt, ++npre) {
+            for (int i = w.k0; i < w.k1 && npre < ST; ++i, ++npre) {
                 const uint32_t a = sbase + npre * L::STAGE, full = smem_addr(&bar_full[npre]);
                 mbar_expect_tx_only(full, weight_bytes());
-                weight_loads(w, kt, a, a + L::A_BYTES, full);
+                weight_loads(w, kstep_of(w, i), a, a + L::A_BYTES, full);
             }
         }
     }
@@ -464,7 +556,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         it.init(p, sched, c, nct);
         Work w;
         while (ok && it.next(p, sched, w)) {
-            for (int kt = w.k0; kt < w.k1; ++kt, ++q_issued) {
+            for (int i = w.k0; i < w.k1; ++i, ++q_issued) {
+                const int kt = kstep_of(w, i);
                 const int stage = q_issued % ST;
                 const uint32_t phase = static_cast<uint32_t>(q_issued / ST) & 1u;
                 const uint32_t a = sbase + stage * L::STAGE, b = a + L::A_BYTES;
@@ -561,7 +654,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint32_t acc_phase = 0;
         bool ok = true;
         const int ldh_r = p.I, ldh_s = p.S * p.I;
-        const int total = sched.prefix[sched.ngroups];
         auto tmem_at = [&](int col) -> uint32_t {
             return tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) + static_cast<uint32_t>(acc * 256 + col);
         };
@@ -603,7 +695,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const bool whole = w.k0 == 0 && w.k1 == w.kt;
                 float* my_slot = nullptr;
                 if (!whole) {
-                    const bool first = range_begin(c, total, nct) >= w.tile_start;
+                    const bool first = it.sk_range_begin(c) >= w.tile_start;
                     my_slot = p.partials + static_cast<size_t>(2 * c + (first ? 0 : 1)) * slot_floats;
                 }
                 for (int ch = 0; ch < nch; ++ch) {
@@ -612,11 +704,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (kG1) tmem_ld16(tmem_at(128 + ch * 16), vb);
                     tmem_ld_wait();
                     if (!whole) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            my_slot[(ch * 16 + j) * BM + r_in] = va[j];
-                            if (kG1) my_slot[(NMAX + ch * 16 + j) * BM + r_in] = vb[j];
-                        }
+                        slot_store16(my_slot + slot_off<NMAX>(0, ch, r_in), va);
+                        if (kG1) slot_store16(my_slot + slot_off<NMAX>(1, ch, r_in), vb);
                         continue;
                     }
 #pragma unroll
@@ -630,45 +719,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (lane == 0) mbar_arrive(smem_addr(&bar_tempty[acc]));
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
-                if (whole) continue;
-                // ---- split tile: the last contributor sums the partials in CTA order
-                const int c_first = cta_of(w.tile_start, total, nct);
-                const int c_last = cta_of(w.tile_start + w.kt - 1, total, nct);
-                int nparts = 0;
-                for (int c2 = c_first; c2 <= c_last; ++c2)
-                    if (range_begin(c2 + 1, total, nct) > range_begin(c2, total, nct)) ++nparts;
-                int32_t* ctr = p.counters + static_cast<size_t>(g) * p.max_tiles + w.n;
-                __threadfence();
-                epi_bar();
-                if (etid == 0) {
-                    const int old = atomicAdd(ctr, 1);
-                    last_sh = (old == nparts - 1);
-                }
-                epi_bar();
-                if (!last_sh) continue;
-                __threadfence();
-                if (etid == 0) *ctr = 0;   // ready for the next call
-                for (int ch = 0; ch < nch; ++ch) {
-                    float va[16], vb[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) { va[j] = 0.f; vb[j] = 0.f; }
-                    for (int c2 = c_first; c2 <= c_last; ++c2) {
-                        const long b2 = range_begin(c2, total, nct);
-                        if (range_begin(c2 + 1, total, nct) <= b2) continue;
-                        const float* sl = p.partials +
-                                          static_cast<size_t>(2 * c2 + (b2 < w.tile_start ? 1 : 0)) * slot_floats;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            va[j] += __ldcg(sl + (ch * 16 + j) * BM + r_in);
-                            if (kG1) vb[j] += __ldcg(sl + (NMAX + ch * 16 + j) * BM + r_in);
-                        }
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int t = ch * 16 + j;
-                        if (t < rows) store_stream(shared, row0, f, t, va[j], kG1 ? vb[j] : 0.f);
-                    }
-                }
+                // a split tile's parts are summed by ffn_finish_kernel after this kernel
             } else {
                 const int rr = w.m0 + r_in;                  // row within the group
                 const bool valid = rr < rows;
@@ -737,16 +788,81 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (threadIdx.x == 32) tstamp(p, MODE, TS_EXIT);
 }
 
+// ------------------------------------------------------------ finish kernel
+// Sums the parts of every tile the streaming GEMM split between CTAs (its
+// contributors wrote fp32 partials and moved on) in CTA order, and applies
+// that GEMM's epilogue: SwiGLU -> h for GEMM1, y for GEMM2, logits for the
+// vocab head.  Running after the GEMM, it reads the partials from a quiet
+// memory system instead of competing with the GEMM's weight stream.  One CTA
+// per (split tile, 16-column chunk); 128 threads = the tile's 128 rows.
+template <int MODE, int NMAX>
+__global__ void __launch_bounds__(BM) ffn_finish_kernel(const Params p) {
+    __shared__ Sched sched;
+    grid_dep_wait();
+    grid_dep_launch();
+    build_schedule<MODE>(p, sched);
+    WorkIter<MODE> it;
+    it.init(p, sched, 0, p.nct);
+    const int nt = sched.tprefix[sched.ngroups];
+    const int first_split = p.nct * (nt / p.nct);
+    const int t = first_split + static_cast<int>(blockIdx.x);
+    if (t >= nt) return;
+    const int g = find_group_tile(sched, t);
+    const int kt = group_ktiles<MODE>(p, g);
+    const int n = t - sched.tprefix[g];
+    const int tile_start = sched.prefix[g] + n * kt;
+    const int c_first = it.sk_cta_of(tile_start), c_last = it.sk_cta_of(tile_start + kt - 1);
+    if (c_first == c_last) return;   // one CTA did the whole tile and stored it
+    const int rows = sched.rows[g], row0 = sched.row0[g];
+    const int ch = blockIdx.y;
+    if (ch * 16 >= rows) return;
+    constexpr bool kG1 = Cfg<MODE>::kG1;
+    const int slot_floats = BM * NMAX * (kG1 ? 2 : 1);
+    const int r = threadIdx.x;
+    auto slot_of = [&](int c2) -> const float* {
+        const int b2 = it.sk_range_begin(c2);
+        if (it.sk_range_begin(c2 + 1) <= b2) return nullptr;   // empty range: not a contributor
+        return p.partials + static_cast<size_t>(2 * c2 + (b2 < tile_start ? 1 : 0)) * slot_floats;
+    };
+    float va[16], vb[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) { va[j] = 0.f; vb[j] = 0.f; }
+    slot_sum16<NMAX>(slot_of, c_first, c_last, 0, ch, r, va);
+    if (kG1) slot_sum16<NMAX>(slot_of, c_first, c_last, 1, ch, r, vb);
+    const bool shared = p.offsets != nullptr && g == p.E;
+    const int f = n * BM + r;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const int tok = ch * 16 + j;
+        if (tok >= rows) break;
+        if (MODE == G1_STREAM) {
+            __nv_bfloat16* dst = shared ? p.h_sh + static_cast<size_t>(tok) * (p.S * p.I) + f
+                                        : p.h_perm + static_cast<size_t>(row0 + tok) * p.I + f;
+            *dst = __float2bfloat16_rn(silu_mul(va[j], vb[j]));
+        } else if (MODE == G2_STREAM) {
+            if (shared) {
+                p.y_sh[static_cast<size_t>(tok) * p.H + f] = va[j];
+            } else if (p.y_bf16) {
+                reinterpret_cast<__nv_bfloat16*>(p.y_perm)[static_cast<size_t>(row0 + tok) * p.H + f] =
+                    __float2bfloat16_rn(va[j]);
+            } else {
+                reinterpret_cast<float*>(p.y_perm)[static_cast<size_t>(row0 + tok) * p.H + f] = va[j];
+            }
+        } else {
+            p.logits[static_cast<size_t>(tok) * p.V + f] = __float2bfloat16_rn(va[j]);
+        }
+    }
+}
+
 // ------------------------------------------------------------ prep kernel
 // Gathers the routed token rows into expert order, pads token operands to
-// whole TMA boxes with zeros, and clears the split-tile counters.
+// whole TMA boxes with zeros.
 __global__ void __launch_bounds__(256) ffn_prep_kernel(const __nv_bfloat16* __restrict__ x,
                                                        const int32_t* __restrict__ perm, int T,
                                                        int H, int rows, int rows_pad,
                                                        __nv_bfloat16* __restrict__ x_perm,
                                                        __nv_bfloat16* __restrict__ x_pad,
-                                                       int t_pad, int32_t* __restrict__ ctr,
-                                                       int nctr, int32_t* status) {
+                                                       int t_pad, int32_t* status) {
     grid_dep_wait();
     grid_dep_launch();
     const int n8 = H / 8;
@@ -774,7 +890,6 @@ __global__ void __launch_bounds__(256) ffn_prep_kernel(const __nv_bfloat16* __re
             reinterpret_cast<uint4*>(x_pad + static_cast<size_t>(r) * H)[c] = val;
         }
     }
-    for (long v = tid; v < nctr; v += stride) ctr[v] = 0;
 }
 
 // ------------------------------------------------------------ host side
@@ -830,13 +945,23 @@ static ms_status launch_gemm(int id, const Maps& maps, const Params& prm, cudaSt
     return launch(id, ffn_gemm_kernel<MODE, NMAX>, dim3(num_sms()), dim3(NTHREADS), L::SMEM, s, maps, prm);
 }
 
+template <int MODE, int NMAX>
+static ms_status launch_stream_n(int id, const Maps& maps, Params prm, cudaStream_t s) {
+    prm.nct = num_sms();
+    ms_status st = launch_gemm<MODE, NMAX>(id, maps, prm, s);
+    if (st != MS_OK) return st;
+    // at most nct - 1 tiles are split; one CTA per (tile, 16-column chunk)
+    return launch(K_FFN_FINISH, ffn_finish_kernel<MODE, NMAX>, dim3(num_sms(), NMAX / 16), dim3(BM), 0, s, prm);
+}
+
+// The streaming GEMM followed by the kernel that finishes its split tiles.
 template <int MODE>
 static ms_status launch_stream(int id, int nmax, const Maps& maps, const Params& prm, cudaStream_t s) {
     switch (nmax) {
-        case 16: return launch_gemm<MODE, 16>(id, maps, prm, s);
-        case 32: return launch_gemm<MODE, 32>(id, maps, prm, s);
-        case 64: return launch_gemm<MODE, 64>(id, maps, prm, s);
-        default: return launch_gemm<MODE, 128>(id, maps, prm, s);
+        case 16: return launch_stream_n<MODE, 16>(id, maps, prm, s);
+        case 32: return launch_stream_n<MODE, 32>(id, maps, prm, s);
+        case 64: return launch_stream_n<MODE, 64>(id, maps, prm, s);
+        default: return launch_stream_n<MODE, 128>(id, maps, prm, s);
     }
 }
 
@@ -852,10 +977,9 @@ static int stream_nmax(int T) {
 struct FfnWs {
     int32_t* status;
     __nv_bfloat16 *x_pad, *x_perm, *h_perm, *h_sh;
-    int32_t* counters;
     float* partials;
     size_t bytes;
-    int t_pad, rows_pad, max_tiles, nctr;
+    int t_pad, rows_pad;
 };
 
 static FfnWs ffn_ws_layout(void* base, int T, int H, int E, int I, int S, int k) {
@@ -870,21 +994,13 @@ static FfnWs ffn_ws_layout(void* base, int T, int H, int E, int I, int S, int k)
     const bool stream = T <= 128;
     w.t_pad = static_cast<int>(align_up(T, BM));
     w.rows_pad = static_cast<int>(align_up(static_cast<size_t>(T) * k, BM));
-    w.max_tiles = 1;
-    {
-        const int cand[3] = {(S > 0 ? S * I : I) / BM, H / BM, I / BM};
-        for (int q = 0; q < 3; ++q) w.max_tiles = cand[q] > w.max_tiles ? cand[q] : w.max_tiles;
-    }
-    const int ngroups = E + (S > 0 ? 1 : 0);
-    w.nctr = 2 * ngroups * w.max_tiles;
     w.status = reinterpret_cast<int32_t*>(take(256));
     w.x_pad = reinterpret_cast<__nv_bfloat16*>(take(stream ? static_cast<size_t>(w.t_pad) * H * 2 : 0));
     w.x_perm = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(w.rows_pad) * H * 2));
     w.h_perm = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(w.rows_pad) * I * 2));
     w.h_sh = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(w.t_pad) * (S > 0 ? S * I : BK) * 2));
-    w.counters = reinterpret_cast<int32_t*>(take(static_cast<size_t>(w.nctr) * 4));
     const size_t slot = static_cast<size_t>(BM) * (stream ? stream_nmax(T) : 16) * 2 * sizeof(float);
-    w.partials = reinterpret_cast<float*>(take(stream ? slot * 2 * num_sms() : 0));
+    w.partials = reinterpret_cast<float*>(take(stream ? slot * 4 * num_sms() : 0));
     w.bytes = off;
     return w;
 }
@@ -900,14 +1016,14 @@ ms_status ffn_launch(const void* x, const int32_t* offsets, const int32_t* perm,
     FfnWs w = ffn_ws_layout(ws, T, H, E, I, S, k);
     const bool stream = T <= 128;
     const int rows = T * k;
-    // 1. gather + pad + clear counters
+    // 1. gather + pad
     {
         const long work = static_cast<long>(w.rows_pad) * (H / 8);
         const int grid = static_cast<int>(work / 256 + 1 < 4L * num_sms() ? work / 256 + 1 : 4L * num_sms());
         ms_status st = launch(K_FFN_PREP, ffn_prep_kernel, dim3(grid), dim3(256), 0, s,
                               reinterpret_cast<const __nv_bfloat16*>(x), perm, T, H, rows, w.rows_pad,
                               w.x_perm, stream ? w.x_pad : static_cast<__nv_bfloat16*>(nullptr), w.t_pad,
-                              w.counters, w.nctr, w.status);
+                              w.status);
         if (st != MS_OK) return st;
     }
     Params prm{};
@@ -921,41 +1037,36 @@ ms_status ffn_launch(const void* x, const int32_t* offsets, const int32_t* perm,
     prm.y_sh = y_sh;
     prm.partials = w.partials;
     prm.status = w.status;
-    prm.max_tiles = w.max_tiles;
     prm.wait_limit_ns = wait_limit_ns();
     prm.dtrace = g_dtrace;
-    const int ngroups = E + (S > 0 ? 1 : 0);
     const uint32_t tok_box = stream ? TOKBOX : BM;
     const void* x_tok_s = stream ? static_cast<const void*>(w.x_pad) : x;
     const int x_rows = stream ? w.t_pad : T;
-    // 2. GEMM1: gate/up + SwiGLU -> h
-    Maps m1{};
+    // 2. GEMM1: gate/up + SwiGLU -> h;  3. GEMM2: down projection -> y_perm, y_shared
+    Maps m1{}, m2{};
     bool ok = make_packed_map(&m1.w_a, wgu, 2 * I, H, E) &&
               make_map(&m1.tok_r, w.x_perm, H, w.rows_pad, 1, tok_box) &&
               make_map(&m1.tok_s, x_tok_s, H, x_rows, 1, tok_box);
     ok = ok && (S > 0 ? make_packed_map(&m1.w_s, wsgu, 2 * I, H, S) : make_packed_map(&m1.w_s, wgu, 2 * I, H, E));
-    if (!ok) return MS_ERR_CUDA;
-    prm.counters = w.counters;
-    ms_status st = stream ? launch_stream<G1_STREAM>(K_GEMM1_STREAM, stream_nmax(T), m1, prm, s)
-                          : launch_gemm<G1_TILED, 16>(K_GEMM1_TILED, m1, prm, s);
-    if (st != MS_OK) return st;
-    // 3. GEMM2: down projection -> y_perm, y_shared
-    Maps m2{};
     const int hs_cols = S > 0 ? S * I : BK;
-    ok = make_packed_map(&m2.w_a, wd, H, I, E) && make_map(&m2.tok_r, w.h_perm, I, w.rows_pad, 1, tok_box) &&
+    ok = ok && make_packed_map(&m2.w_a, wd, H, I, E) && make_map(&m2.tok_r, w.h_perm, I, w.rows_pad, 1, tok_box) &&
          make_map(&m2.tok_s, w.h_sh, hs_cols, w.t_pad, 1, tok_box);
     ok = ok && (S > 0 ? make_packed_map(&m2.w_s, wsd, H, I, S) : make_packed_map(&m2.w_s, wd, H, I, E));
     if (!ok) return MS_ERR_CUDA;
-    prm.counters = w.counters + ngroups * w.max_tiles;
-    return stream ? launch_stream<G2_STREAM>(K_GEMM2_STREAM, stream_nmax(T), m2, prm, s)
-                  : launch_gemm<G2_TILED, 16>(K_GEMM2_TILED, m2, prm, s);
+    if (stream) {
+        ms_status st1 = launch_stream<G1_STREAM>(K_GEMM1_STREAM, stream_nmax(T), m1, prm, s);
+        if (st1 != MS_OK) return st1;
+        return launch_stream<G2_STREAM>(K_GEMM2_STREAM, stream_nmax(T), m2, prm, s);
+    }
+    ms_status st = launch_gemm<G1_TILED, 16>(K_GEMM1_TILED, m1, prm, s);
+    if (st != MS_OK) return st;
+    return launch_gemm<G2_TILED, 16>(K_GEMM2_TILED, m2, prm, s);
 }
 
 // ------------------------------------------------------------ vocab head
 struct LmWs {
     int32_t* status;
     __nv_bfloat16* x_pad;
-    int32_t* counters;
     float* partials;
     size_t bytes;
 };
@@ -971,7 +1082,6 @@ static LmWs lm_ws_layout(void* base, int H, int V) {
     };
     w.status = reinterpret_cast<int32_t*>(take(256));
     w.x_pad = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(BM) * H * 2));
-    w.counters = reinterpret_cast<int32_t*>(take(static_cast<size_t>(V / BM) * 4));
     w.partials = reinterpret_cast<float*>(take(static_cast<size_t>(BM) * 128 * sizeof(float) * 2 * num_sms()));
     w.bytes = off;
     return w;
@@ -987,7 +1097,7 @@ ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* l
         const __nv_bfloat16* xc = reinterpret_cast<const __nv_bfloat16*>(x) + static_cast<size_t>(t0) * H;
         ms_status st = launch(K_FFN_PREP, ffn_prep_kernel, dim3(2 * num_sms()), dim3(256), 0, s, xc,
                               static_cast<const int32_t*>(nullptr), tc, H, 0, 0,
-                              static_cast<__nv_bfloat16*>(nullptr), w.x_pad, BM, w.counters, V / BM, w.status);
+                              static_cast<__nv_bfloat16*>(nullptr), w.x_pad, BM, w.status);
         if (st != MS_OK) return st;
         Maps m{};
         bool ok = make_packed_map(&m.w_a, wlm, V, H, 1) && make_packed_map(&m.w_s, wlm, V, H, 1) &&
@@ -999,9 +1109,7 @@ ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* l
         prm.offsets = nullptr;
         prm.logits = reinterpret_cast<__nv_bfloat16*>(logits) + static_cast<size_t>(t0) * V;
         prm.partials = w.partials;
-        prm.counters = w.counters;
         prm.status = w.status;
-        prm.max_tiles = V / BM;
         prm.wait_limit_ns = wait_limit_ns();
         prm.dtrace = g_dtrace;
         st = launch_stream<LM_STREAM>(K_LM_HEAD, stream_nmax(tc), m, prm, s);

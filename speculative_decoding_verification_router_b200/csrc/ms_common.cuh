@@ -24,6 +24,7 @@ enum KernelId : int {
     K_GEMM2_STREAM,
     K_GEMM1_TILED,
     K_GEMM2_TILED,
+    K_FFN_FINISH,
     K_LM_HEAD,
     K_COMBINE,
     K_VERIFY_PARTIAL,

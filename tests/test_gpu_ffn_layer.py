@@ -211,6 +211,6 @@ def test_trace_records_kernels(ms):
         ms.trace_disable()
         ms.trace_reset()
     names = [n for n, _ in recs]
-    assert names == ["route_cluster", "permute_scatter", "ffn_prep", "gemm1_stream", "gemm2_stream",
-                     "combine"], names
+    assert names == ["route_cluster", "permute_scatter", "ffn_prep", "gemm1_stream", "ffn_finish", "gemm2_stream",
+                     "ffn_finish", "combine"], names
     assert all(t > 0 for _, t in recs)
