@@ -123,6 +123,9 @@ MS_API ms_status moe_pack_weights(const void* w, int n, int rows, int cols, void
  * y_shared: [T,H] fp32 (may be NULL iff S == 0).
  * Tensor-core grouped GEMMs (tcgen05 + TMEM, TMA-fed).  T <= 128 uses a
  * weight-streaming schedule balanced over all SMs; larger T a tiled one.
+ * expert_offsets must describe groups inside [0, T*k) of at most T rows
+ * each (a token reaches an expert at most once); a group that does not is
+ * skipped and flagged MS_ERR_DEVICE_INDEX in the status word.
  * Scratch: moe_expert_ffn_workspace_size(...) bytes; the status word of
  * the bounded waits lives at its start (see ms_device_status). */
 MS_API size_t moe_expert_ffn_workspace_size(int T, int H, int E, int I, int S, int k);
@@ -221,13 +224,16 @@ MS_API ms_status ms_debug_bounded_wait(const int32_t* flag, int32_t expect, int3
                                 void* stream);
 
 /* In-kernel timeline of the tensor-core GEMMs: while a device buffer of at
- * least 5*256*8 uint64 (80 KB) is set, every CTA of every GEMM launch writes
- * globaltimer stamps (ns) to buf[(mode*256 + cta)*8 + slot], mode 0..4 =
+ * least 8*256*8 uint64 (128 KB) is set, every CTA of every GEMM launch writes
+ * globaltimer stamps (ns) to buf[(row*256 + cta)*8 + slot], row 0..4 =
  * GEMM1 streaming, GEMM2 streaming, vocab head, GEMM1 tiled, GEMM2 tiled;
  * slot 0 entry, 1 schedule built, 2 setup done (after the wait on the previous
  * kernel), 3 first stage of data ready, 4 last MMA issued, 5 epilogue done,
- * 6 loads drained, 7 exit.  A later launch of the same mode overwrites.
- * buf = NULL disables it.  For profiling only. */
+ * 6 loads drained, 7 exit.  Rows 5..7 hold the split-tile finish kernels of
+ * the three streaming modes (CTA = blockIdx.x of the first column chunk):
+ * slot 0 entry, 1 after the wait on the GEMM, 2 schedule built, 7 exit (only
+ * CTAs that finish a tile write slot 7).  A later launch of the same kind
+ * overwrites.  buf = NULL disables it.  For profiling only. */
 MS_API ms_status ms_set_device_trace(void* buf, size_t bytes);
 
 /* Launch tracing: when enabled, every kernel this library launches is

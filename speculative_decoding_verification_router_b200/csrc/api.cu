@@ -197,7 +197,7 @@ ms_status ms_device_status(void* ws, void* stream) {
 void ms_set_wait_limit_ns(uint64_t ns) { ms::g_wait_limit_ns = ns; }
 
 ms_status ms_set_device_trace(void* buf, size_t bytes) {
-    if (buf && bytes < static_cast<size_t>(5) * 256 * 8 * sizeof(uint64_t)) return MS_ERR_WORKSPACE;
+    if (buf && bytes < static_cast<size_t>(8) * 256 * 8 * sizeof(uint64_t)) return MS_ERR_WORKSPACE;
     ms::set_device_trace(buf);
     return MS_OK;
 }

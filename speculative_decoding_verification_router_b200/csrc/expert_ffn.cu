@@ -150,12 +150,12 @@ __device__ __forceinline__ int group_ntiles(const Params& p, int g) {
     return p.H / p.bn;   // G2_TILED
 }
 
-template <int MODE>
-__device__ void build_schedule(const Params& p, Sched& s) {
+template <int MODE, int NT>
+__device__ void build_schedule_n(const Params& p, Sched& s) {
     const int tid = threadIdx.x;
     s.ngroups = p.offsets == nullptr ? 1 : p.E + (p.S > 0 ? 1 : 0);
     const int ng = s.ngroups;
-    for (int g = tid; g < ng; g += NTHREADS) {
+    for (int g = tid; g < ng; g += NT) {
         int rows, row0;
         if (p.offsets == nullptr) {
             rows = p.T;
@@ -163,7 +163,9 @@ __device__ void build_schedule(const Params& p, Sched& s) {
         } else if (g < p.E) {
             row0 = __ldg(p.offsets + g);
             rows = __ldg(p.offsets + g + 1) - row0;
-            if (rows < 0 || row0 < 0 || row0 + rows > p.T * p.k) {
+            // a token reaches an expert at most once, so no group exceeds T
+            // rows; the streaming schedule's token buffers hold T rows only
+            if (rows < 0 || row0 < 0 || row0 + rows > p.T * p.k || (Cfg<MODE>::kStream && rows > p.T)) {
                 report_status(p.status, MS_ERR_DEVICE_INDEX);
                 rows = 0;
             }
@@ -190,6 +192,9 @@ __device__ void build_schedule(const Params& p, Sched& s) {
     else if (tid < 64) warp_scan_groups(s.tprefix, ng, tid - 32);
     __syncthreads();
 }
+
+template <int MODE>
+__device__ void build_schedule(const Params& p, Sched& s) { build_schedule_n<MODE, NTHREADS>(p, s); }
 
 // largest g with prefix[g] <= pos (g < ngroups); groups with no work have
 // prefix[g] == prefix[g+1] and are never returned for pos < total.
@@ -253,15 +258,25 @@ __device__ __forceinline__ int find_group_tile(const Sched& s, int t) {
     return lo;
 }
 
+// Whole tiles per CTA on the streaming schedule: every full round of tiles
+// but the last, so that the split region holds the last nct .. 2 nct - 1
+// tiles (all of them when NT < nct).  Each CTA's split range is then at least
+// one tile long and a split tile has two contributors, three at most, so the
+// finish kernel sums it in one round of loads.
+__device__ __forceinline__ int dp_tiles_per_cta(int nt, int nct) {
+    const int q = nt / nct;
+    return q > 0 ? q - 1 : 0;
+}
+
 template <int MODE>
 struct WorkIter {
     // Streaming ("data-parallel + stream-K", split part first): with NT output
-    // tiles in group order and nct CTAs, CTA c owns the D = NT / nct whole
-    // tiles [c*D, c*D + D); the k-steps of the remaining NT - nct*D tiles at the
-    // end of the order (the split region) are divided into nct equal ranges.
-    // A CTA walks its split range first and its whole tiles last, so every
-    // tile shared between CTAs is finished (and its fix-up done) early and the
-    // kernel ends on whole tiles, whose epilogue is a plain store.
+    // tiles in group order and nct CTAs, CTA c owns the D = dp_tiles_per_cta
+    // whole tiles [c*D, c*D + D); the k-steps of the remaining NT - nct*D
+    // tiles at the end of the order (the split region) are divided into nct
+    // equal ranges.  A CTA walks its split range first and its whole tiles
+    // last.  Contributors to a split tile store fp32 partials; the finish
+    // kernel that follows the GEMM sums them and applies the epilogue.
     // Tiled: tiles c, c + nct, ... (round robin).
     int c, nct, state, pos, re, dp_next, dp_end, t, total;
     int sk_begin, sk_total;   // split region in absolute k-step positions
@@ -272,7 +287,7 @@ struct WorkIter {
         total = s.prefix[s.ngroups];
         if (Cfg<MODE>::kStream) {
             const int nt = s.tprefix[s.ngroups];
-            const int D = nt / nct;
+            const int D = dp_tiles_per_cta(nt, nct);
             dp_next = c * D;
             dp_end = dp_next + D;
             const int first_split_tile = nct * D;
@@ -375,36 +390,46 @@ __device__ __forceinline__ void slot_store16(float* dst, const float (&v)[16]) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
-// v += the 16 values of every contributor's slot, contributors in CTA order;
-// loads of up to four contributors are issued before their additions.
-template <int NMAX, typename SlotOf>
-__device__ __forceinline__ void slot_sum16(SlotOf slot_of, int c_first, int c_last, int half, int ch, int r,
-                                           float (&v)[16]) {
+// va (and vb, for GEMM1's second half) += the first 4*NQ values of every
+// contributor's slot of chunk ch, row r, contributors in CTA order.  The loads
+// of 8/NQ contributors (both halves) are issued before any addition, so the
+// usual two or three contributors cost one round trip.
+template <int NMAX, int NQ, bool G1, typename SlotOf>
+__device__ __forceinline__ void slot_sum(SlotOf slot_of, int c_first, int c_last, int ch, int r,
+                                         float (&va)[16], float (&vb)[16]) {
+    constexpr int CB = 8 / NQ;
     int c2 = c_first;
     while (true) {
-        const float* src[4];
+        const float* src[CB];
         int nb = 0;
-        for (; c2 <= c_last && nb < 4; ++c2) {
+        for (; c2 <= c_last && nb < CB; ++c2) {
             const float* sl = slot_of(c2);
-            if (sl) src[nb++] = sl + slot_off<NMAX>(half, ch, r);
+            if (sl) src[nb++] = sl;
         }
         if (nb == 0) break;
-        float4 x[4][4];
+        float4 xa[CB][NQ], xb[CB][NQ];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < CB; ++u)
             if (u < nb) {
+                const float4* pa = reinterpret_cast<const float4*>(src[u] + slot_off<NMAX>(0, ch, r));
+                const float4* pb = reinterpret_cast<const float4*>(src[u] + slot_off<NMAX>(1, ch, r));
 #pragma unroll
-                for (int q = 0; q < 4; ++q) x[u][q] = __ldcg(reinterpret_cast<const float4*>(src[u]) + q);
+                for (int q = 0; q < NQ; ++q) {
+                    xa[u][q] = __ldcg(pa + q);
+                    if (G1) xb[u][q] = __ldcg(pb + q);
+                }
             }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < CB; ++u)
             if (u < nb) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    v[4 * q] += x[u][q].x;
-                    v[4 * q + 1] += x[u][q].y;
-                    v[4 * q + 2] += x[u][q].z;
-                    v[4 * q + 3] += x[u][q].w;
+                for (int q = 0; q < NQ; ++q) {
+                    va[4 * q] += xa[u][q].x; va[4 * q + 1] += xa[u][q].y;
+                    va[4 * q + 2] += xa[u][q].z; va[4 * q + 3] += xa[u][q].w;
+                    if (G1) {
+                        vb[4 * q] += xb[u][q].x; vb[4 * q + 1] += xb[u][q].y;
+                        vb[4 * q + 2] += xb[u][q].z; vb[4 * q + 3] += xb[u][q].w;
+                    }
                 }
             }
     }
@@ -793,18 +818,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // contributors wrote fp32 partials and moved on) in CTA order, and applies
 // that GEMM's epilogue: SwiGLU -> h for GEMM1, y for GEMM2, logits for the
 // vocab head.  Running after the GEMM, it reads the partials from a quiet
-// memory system instead of competing with the GEMM's weight stream.  One CTA
-// per (split tile, 16-column chunk); 128 threads = the tile's 128 rows.
+// memory system instead of competing with the GEMM's weight stream.
+// One CTA per (split tile, 16-column chunk); 128 threads = the tile's rows.
+// timeline row of the finish kernel that follows GEMM mode MODE
+template <int MODE>
+__device__ __forceinline__ void fin_stamp(const Params& p, int slot) {
+    if (blockIdx.y == 0 && threadIdx.x == 0) tstamp(p, 5 + MODE, slot);
+}
+
+constexpr int FIN_THREADS = BM;
+
 template <int MODE, int NMAX>
-__global__ void __launch_bounds__(BM) ffn_finish_kernel(const Params p) {
+__global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p) {
     __shared__ Sched sched;
+    fin_stamp<MODE>(p, TS_ENTRY);
+    // The offsets come from a kernel at least two launches back, which every
+    // kernel of this library waits for before it lets its successor start:
+    // they may be read before this launch's own wait.
+    build_schedule_n<MODE, FIN_THREADS>(p, sched);
     grid_dep_wait();
     grid_dep_launch();
-    build_schedule<MODE>(p, sched);
+    fin_stamp<MODE>(p, TS_SCHEDULE);
     WorkIter<MODE> it;
     it.init(p, sched, 0, p.nct);
     const int nt = sched.tprefix[sched.ngroups];
-    const int first_split = p.nct * (nt / p.nct);
+    const int first_split = p.nct * dp_tiles_per_cta(nt, p.nct);
     const int t = first_split + static_cast<int>(blockIdx.x);
     if (t >= nt) return;
     const int g = find_group_tile(sched, t);
@@ -826,9 +864,12 @@ __global__ void __launch_bounds__(BM) ffn_finish_kernel(const Params p) {
     };
     float va[16], vb[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) { va[j] = 0.f; vb[j] = 0.f; }
-    slot_sum16<NMAX>(slot_of, c_first, c_last, 0, ch, r, va);
-    if (kG1) slot_sum16<NMAX>(slot_of, c_first, c_last, 1, ch, r, vb);
+    for (int j = 0; j < 16; ++j) va[j] = vb[j] = 0.f;
+    const int rc = rows - ch * 16;   // tokens of this chunk (only those are read)
+    if (rc <= 4) slot_sum<NMAX, 1, kG1>(slot_of, c_first, c_last, ch, r, va, vb);
+    else if (rc <= 8) slot_sum<NMAX, 2, kG1>(slot_of, c_first, c_last, ch, r, va, vb);
+    else slot_sum<NMAX, 4, kG1>(slot_of, c_first, c_last, ch, r, va, vb);
+    fin_stamp<MODE>(p, TS_FIRST_DATA);
     const bool shared = p.offsets != nullptr && g == p.E;
     const int f = n * BM + r;
 #pragma unroll
@@ -852,6 +893,7 @@ __global__ void __launch_bounds__(BM) ffn_finish_kernel(const Params p) {
             p.logits[static_cast<size_t>(tok) * p.V + f] = __float2bfloat16_rn(va[j]);
         }
     }
+    fin_stamp<MODE>(p, TS_EXIT);
 }
 
 // ------------------------------------------------------------ prep kernel
@@ -950,8 +992,9 @@ static ms_status launch_stream_n(int id, const Maps& maps, Params prm, cudaStrea
     prm.nct = num_sms();
     ms_status st = launch_gemm<MODE, NMAX>(id, maps, prm, s);
     if (st != MS_OK) return st;
-    // at most nct - 1 tiles are split; one CTA per (tile, 16-column chunk)
-    return launch(K_FFN_FINISH, ffn_finish_kernel<MODE, NMAX>, dim3(num_sms(), NMAX / 16), dim3(BM), 0, s, prm);
+    // fewer than 2 nct tiles are split; one CTA per (tile, 16-column chunk)
+    return launch(K_FFN_FINISH, ffn_finish_kernel<MODE, NMAX>, dim3(2 * num_sms(), NMAX / 16), dim3(FIN_THREADS),
+                  0, s, prm);
 }
 
 // The streaming GEMM followed by the kernel that finishes its split tiles.

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <utility>
 
 #include "moespec.h"
@@ -41,6 +42,16 @@ void trace_mark(int id, cudaStream_t s, bool after);
 uint64_t wait_limit_ns();
 void set_cuda_error(cudaError_t e);
 
+// Programmatic dependent launch is on unless MOESPEC_NO_PDL=1 (a measurement
+// knob: kernels are correct either way, since each waits for its predecessor).
+inline int pdl_allowed() {
+    static const int on = [] {
+        const char* e = getenv("MOESPEC_NO_PDL");
+        return (e && e[0] == '1') ? 0 : 1;
+    }();
+    return on;
+}
+
 // Launch `kernel` with programmatic stream serialisation allowed, so that it
 // may start while the previous kernel on the stream finishes; the kernel
 // itself calls grid_dep_wait() before touching dependent memory.
@@ -54,7 +65,7 @@ inline ms_status launch(int id, void (*kernel)(KArgs...), dim3 grid, dim3 block,
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_allowed();
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     trace_mark(id, s, false);
@@ -78,7 +89,7 @@ inline ms_status launch_cluster(int id, void (*kernel)(KArgs...), dim3 grid, dim
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_allowed();
     attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = cluster_x;
     attr[1].val.clusterDim.y = 1;

@@ -48,22 +48,29 @@ __global__ void __launch_bounds__(PM_THREADS) permute_count_kernel(const int32_t
         hist[static_cast<size_t>(blockIdx.x) * E + e] = cnt[e];
 }
 
-// Stable scatter.  With one block the block computes the offsets itself;
-// with several, `hist` holds every block's histogram from permute_count_kernel.
-__global__ void __launch_bounds__(PM_THREADS) permute_scatter_kernel(
-    const int32_t* __restrict__ idx, int n, int k, int E, const int32_t* __restrict__ hist,
-    int nblocks, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
-    int32_t* __restrict__ slot_of, int32_t* status) {
-    __shared__ int32_t wcnt[PM_WARPS][PM_MAX_E];   // per-warp counts, then per-warp bases
-    __shared__ int32_t base[PM_MAX_E];
-    grid_dep_wait();
-    grid_dep_launch();
+// Ranks of one block's chunk of (token, slot) pairs.  On return ex[r] is the
+// expert of pair wbegin + 32 r + lane (-1 past the end or when invalid) and
+// pos[r] its row in expert order.  With nblocks > 1, `hist` holds every block's
+// histogram from permute_count_kernel; with one block the chunk is the whole
+// input and the block computes the offsets itself.  Block `chunk` == 0 writes
+// `offsets` when it is non-null.
+struct SortSmem {
+    int32_t wcnt[PM_WARPS][PM_MAX_E];   // per-warp counts, then per-warp bases
+    int32_t base[PM_MAX_E];
+    int32_t before[PM_MAX_E];
+};
+
+__device__ __forceinline__ void chunk_ranks(const int32_t* __restrict__ idx, int n, int E,
+                                            const int32_t* __restrict__ hist, int nblocks, int chunk,
+                                            int32_t* __restrict__ offsets, SortSmem& sm,
+                                            int (&ex)[PM_PER_LANE], int (&pos)[PM_PER_LANE],
+                                            int32_t* status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int i = threadIdx.x; i < PM_WARPS * PM_MAX_E; i += PM_THREADS) (&wcnt[0][0])[i] = 0;
+    for (int i = threadIdx.x; i < PM_WARPS * PM_MAX_E; i += PM_THREADS) (&sm.wcnt[0][0])[i] = 0;
     __syncthreads();
 
-    const int wbegin = blockIdx.x * PM_CHUNK + warp * PM_PER_WARP;
-    int ex[PM_PER_LANE], rk[PM_PER_LANE];
+    const int wbegin = chunk * PM_CHUNK + warp * PM_PER_WARP;
+    int rk[PM_PER_LANE];
 #pragma unroll
     for (int r = 0; r < PM_PER_LANE; ++r) {
         const int i = wbegin + r * 32 + lane;
@@ -74,9 +81,9 @@ __global__ void __launch_bounds__(PM_THREADS) permute_scatter_kernel(
         }
         const uint32_t peers = __match_any_sync(0xffffffffu, e);
         int rank = 0;
-        if (e >= 0) rank = wcnt[warp][e] + __popc(peers & lanemask_lt());
+        if (e >= 0) rank = sm.wcnt[warp][e] + __popc(peers & lanemask_lt());
         __syncwarp();
-        if (e >= 0 && (peers & lanemask_lt()) == 0) wcnt[warp][e] += __popc(peers);
+        if (e >= 0 && (peers & lanemask_lt()) == 0) sm.wcnt[warp][e] += __popc(peers);
         __syncwarp();
         ex[r] = e;
         rk[r] = rank;
@@ -86,33 +93,32 @@ __global__ void __launch_bounds__(PM_THREADS) permute_scatter_kernel(
     for (int e = threadIdx.x; e < E; e += PM_THREADS) {
         int run = 0;
         for (int w = 0; w < PM_WARPS; ++w) {
-            const int c = wcnt[w][e];
-            wcnt[w][e] = run;
+            const int c = sm.wcnt[w][e];
+            sm.wcnt[w][e] = run;
             run += c;
         }
-        base[e] = run;     // block total for now
+        sm.base[e] = run;     // block total for now
     }
     __syncthreads();
     // global base of expert e for this block:
     //   sum_{e'<e} total[e'] + sum_{b'<b} hist[b'][e]
-    __shared__ int32_t before[PM_MAX_E];
     if (nblocks > 1) {
         for (int e = warp; e < E; e += PM_WARPS) {
             int tot = 0, bef = 0;
             for (int b = lane; b < nblocks; b += 32) {
                 const int h = hist[static_cast<size_t>(b) * E + e];
                 tot += h;
-                if (b < static_cast<int>(blockIdx.x)) bef += h;
+                if (b < chunk) bef += h;
             }
             tot = __reduce_add_sync(0xffffffffu, tot);
             bef = __reduce_add_sync(0xffffffffu, bef);
             if (lane == 0) {
-                base[e] = tot;
-                before[e] = bef;
+                sm.base[e] = tot;
+                sm.before[e] = bef;
             }
         }
     } else {
-        for (int e = threadIdx.x; e < E; e += PM_THREADS) before[e] = 0;
+        for (int e = threadIdx.x; e < E; e += PM_THREADS) sm.before[e] = 0;
     }
     __syncthreads();
     if (warp == 0) {
@@ -123,7 +129,7 @@ __global__ void __launch_bounds__(PM_THREADS) permute_scatter_kernel(
         int sum = 0;
 #pragma unroll
         for (int q = 0; q < kPer; ++q) {
-            loc[q] = (e0 + q < E) ? base[e0 + q] : 0;
+            loc[q] = (e0 + q < E) ? sm.base[e0 + q] : 0;
             sum += loc[q];
         }
         int incl = sum;
@@ -137,22 +143,38 @@ __global__ void __launch_bounds__(PM_THREADS) permute_scatter_kernel(
         for (int q = 0; q < kPer; ++q) {
             const int e = e0 + q;
             if (e < E) {
-                if (blockIdx.x == 0) offsets[e] = run;
-                base[e] = run + before[e];
+                if (offsets && chunk == 0) offsets[e] = run;
+                sm.base[e] = run + sm.before[e];
             }
             run += loc[q];
         }
-        if (blockIdx.x == 0 && lane == 31) offsets[E] = incl;
+        if (offsets && chunk == 0 && lane == 31) offsets[E] = incl;
     }
     __syncthreads();
 #pragma unroll
     for (int r = 0; r < PM_PER_LANE; ++r) {
         const int e = ex[r];
-        if (e < 0) continue;
-        const int i = wbegin + r * 32 + lane;
-        const int pos = base[e] + wcnt[warp][e] + rk[r];
-        perm_token[pos] = i / k;
-        slot_of[i] = pos;
+        pos[r] = e < 0 ? -1 : sm.base[e] + sm.wcnt[warp][e] + rk[r];
+    }
+}
+
+// Stable scatter of one chunk per block.
+__global__ void __launch_bounds__(PM_THREADS) permute_scatter_kernel(
+    const int32_t* __restrict__ idx, int n, int k, int E, const int32_t* __restrict__ hist,
+    int nblocks, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
+    int32_t* __restrict__ slot_of, int32_t* status) {
+    __shared__ SortSmem sm;
+    grid_dep_wait();
+    grid_dep_launch();
+    int ex[PM_PER_LANE], pos[PM_PER_LANE];
+    chunk_ranks(idx, n, E, hist, nblocks, static_cast<int>(blockIdx.x), offsets, sm, ex, pos, status);
+    const int wbegin = blockIdx.x * PM_CHUNK + (threadIdx.x >> 5) * PM_PER_WARP + (threadIdx.x & 31);
+#pragma unroll
+    for (int r = 0; r < PM_PER_LANE; ++r) {
+        if (ex[r] < 0) continue;
+        const int i = wbegin + r * 32;
+        perm_token[pos[r]] = i / k;
+        slot_of[i] = pos[r];
     }
 }
 

@@ -285,7 +285,7 @@ def debug_bounded_wait(flag: torch.Tensor, expect: int, status: torch.Tensor, st
 
 
 def set_device_trace(buf: Optional[torch.Tensor]):
-    """Point the GEMMs' per-CTA timeline at `buf` (uint64 tensor, >= 5*256*8), or None to stop."""
+    """Point the GEMMs' per-CTA timeline at `buf` (uint64 tensor, >= 8*256*8), or None to stop."""
     if buf is None:
         _check(_lib.ms_set_device_trace(None, 0), "ms_set_device_trace")
     else:

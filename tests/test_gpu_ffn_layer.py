@@ -62,6 +62,25 @@ def test_expert_ffn_is_deterministic(ms):
     assert torch.equal(y1, y2) and torch.equal(s1, s2)
 
 
+def test_expert_ffn_flags_oversized_group(ms):
+    # offsets that give one expert more than T rows (a token routed to it
+    # twice) are rejected on the device: the group is skipped and flagged,
+    # the other groups and the shared expert are still computed
+    shp = synth.TINY
+    T, k, E = shp.T, shp.k, shp.E
+    lw = synth.layer_weights(shp, 0)
+    wgu, wd, wsgu, wsd = _weights_dev(lw)
+    xb = synth.normal_bf16(0, "oversized_group_x", (T, shp.H), 1.0)
+    off = np.full(E + 1, T * k, np.int32)
+    off[0] = 0
+    perm = (np.arange(T * k) % T).astype(np.int32)
+    ws = ms.Workspace(ms.expert_ffn_workspace_size(T, shp.H, E, shp.I, shp.S, k))
+    y, ysh = ms.expert_ffn(dev(xb), dev(off), dev(perm), wgu, wd, wsgu, wsd, k, ws=ws)
+    assert ms.device_status(ws) == -6
+    rs = oracle.expert_ffn_shared(oracle.widen_bf16(xb), lw.ws_gate_up, lw.ws_down)
+    assert_close(host(ysh), rs, what="y_shared beside a rejected group")
+
+
 @pytest.mark.parametrize("T", [129, 300])
 def test_expert_ffn_tiled_ragged(ms, T):
     # the tiled (large-T) schedule on small shapes, with a ragged last tile
