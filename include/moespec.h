@@ -230,9 +230,9 @@ MS_API ms_status ms_debug_bounded_wait(const int32_t* flag, int32_t expect, int3
  * slot 0 entry, 1 schedule built, 2 setup done (after the wait on the previous
  * kernel), 3 first stage of data ready, 4 last MMA issued, 5 epilogue done,
  * 6 loads drained, 7 exit.  Rows 5..7 hold the split-tile finish kernels of
- * the three streaming modes (CTA = blockIdx.x of the first column chunk):
- * slot 0 entry, 1 after the wait on the GEMM, 2 schedule built, 7 exit (only
- * CTAs that finish a tile write slot 7).  A later launch of the same kind
+ * the three streaming modes (CTA = blockIdx.x < 256 of the first column
+ * chunk): slot 0 entry, 1 after the wait on the GEMM, 3 partials summed, 7
+ * exit (only CTAs that finish a tile write slots 3 and 7).  A later launch of the same kind
  * overwrites.  buf = NULL disables it.  For profiling only. */
 MS_API ms_status ms_set_device_trace(void* buf, size_t bytes);
 

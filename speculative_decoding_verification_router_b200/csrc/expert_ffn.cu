@@ -41,12 +41,16 @@ constexpr int TOKBOX = 16;               // token rows per TMA box (streaming)
 constexpr int NTHREADS = 192;
 constexpr int MAX_GROUPS = 257;
 constexpr int TMEM_COLS = 512;
-#ifndef MS_SMEM_BUDGET_KB
-#define MS_SMEM_BUDGET_KB 140
+#ifndef MS_WEIGHT_BUDGET_KB
+#define MS_WEIGHT_BUDGET_KB 128
 #endif
-// Shared memory for pipeline stages.  More stages means more bytes in flight
-// per SM; beyond what saturates HBM they only lengthen the memory queues.
-constexpr int SMEM_BUDGET = MS_SMEM_BUDGET_KB * 1024;
+// Streaming schedule: weight bytes in flight per SM (pipeline stages x the
+// weight part of a stage).  About 128 KB saturates HBM with 32 KB stages;
+// more only lengthens the memory queues and delays the loads a CTA waits for.
+constexpr int WEIGHT_BUDGET = MS_WEIGHT_BUDGET_KB * 1024;
+// Shared memory for the stages of any schedule (the tiled one is bounded by
+// this alone).
+constexpr int SMEM_CAP = 200 * 1024;
 
 enum Mode : int { G1_STREAM = 0, G2_STREAM = 1, LM_STREAM = 2, G1_TILED = 3, G2_TILED = 4 };
 
@@ -77,21 +81,30 @@ struct Params {
 // Timeline slots written per CTA when a device trace buffer is set.
 enum TraceSlot { TS_ENTRY = 0, TS_SCHEDULE, TS_SETUP, TS_FIRST_DATA, TS_LAST_MMA, TS_EPI_DONE, TS_PRODUCER_DONE, TS_EXIT };
 __device__ __forceinline__ void tstamp(const Params& p, int mode, int slot) {
-    if (p.dtrace) p.dtrace[(static_cast<size_t>(mode) * 256 + blockIdx.x) * 8 + slot] = global_ns();
+    if (p.dtrace && blockIdx.x < 256) p.dtrace[(static_cast<size_t>(mode) * 256 + blockIdx.x) * 8 + slot] = global_ns();
 }
 
 template <int MODE>
 struct Cfg {
     static constexpr bool kStream = MODE <= LM_STREAM;
     static constexpr bool kG1 = MODE == G1_STREAM || MODE == G1_TILED;
+    // 64-wide k-blocks per pipeline stage (one schedule k-step).  GEMM1's
+    // streaming stage already carries two weight tiles (gate and up rows);
+    // the single-operand streaming GEMMs take two consecutive k-blocks, which
+    // are one contiguous 32 KB in the packed layout: per-stage costs
+    // (barrier round trips, TMA issue) are paid per 32 KB, not per 16 KB.
+    static constexpr int kSub = (MODE == G2_STREAM || MODE == LM_STREAM) ? 2 : 1;
 };
 
 template <int MODE, int NMAX>
 struct Layout {
-    static constexpr int A_BYTES = Cfg<MODE>::kStream ? (Cfg<MODE>::kG1 ? 2 : 1) * TILE_BYTES : TILE_BYTES;
-    static constexpr int B_BYTES = Cfg<MODE>::kStream ? NMAX * BK * 2 : 2 * TILE_BYTES;
+    static constexpr int A_BYTES =
+        Cfg<MODE>::kStream ? (Cfg<MODE>::kG1 ? 2 : Cfg<MODE>::kSub) * TILE_BYTES : TILE_BYTES;
+    static constexpr int B_BYTES = Cfg<MODE>::kStream ? Cfg<MODE>::kSub * NMAX * BK * 2 : 2 * TILE_BYTES;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE;
+    static constexpr int BY_WEIGHTS = Cfg<MODE>::kStream ? WEIGHT_BUDGET / A_BYTES : 8;
+    static constexpr int BY_SMEM = SMEM_CAP / STAGE;
+    static constexpr int STAGES_RAW = BY_WEIGHTS < BY_SMEM ? BY_WEIGHTS : BY_SMEM;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static constexpr int SMEM = STAGES * STAGE + 1024;
     static_assert(STAGE % 1024 == 0, "stage buffers must stay 1024-byte aligned");
@@ -137,8 +150,9 @@ __device__ __forceinline__ void warp_scan_groups(int* a, int n, int lane) {
 template <int MODE>
 __device__ __forceinline__ int group_ktiles(const Params& p, int g) {
     const bool shared = p.offsets != nullptr && g == p.E;
-    if (MODE == G1_STREAM || MODE == G1_TILED || MODE == LM_STREAM) return p.H / BK;
-    return (shared ? p.S * p.I : p.I) / BK;   // GEMM2: K = intermediate width
+    constexpr int KS = BK * Cfg<MODE>::kSub;   // k per schedule step
+    if (MODE == G1_STREAM || MODE == G1_TILED || MODE == LM_STREAM) return p.H / KS;
+    return (shared ? p.S * p.I : p.I) / KS;   // GEMM2: K = intermediate width
 }
 
 template <int MODE>
@@ -377,19 +391,54 @@ __device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, uint64_t
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
-// Partial-sum slot of a split tile: [half][chunk][row][16].  A thread's 16
-// values of one chunk are 64 contiguous bytes (four 16-byte accesses) and a
-// warp's 32 rows 2 KB, so contributors write and the finisher reads with
-// full-width vector accesses.
+// Partial-sum slot of a split tile.  GEMM1 (gate and up halves):
+// [half][chunk][row][16], so a thread's 16 values of one chunk are 64
+// contiguous bytes and contributors write and the finisher reads with
+// full-width vector accesses.  GEMM2 and the vocab head (one half):
+// [column][row], so the 4 or 8 consecutive output features of one token that
+// the combine kernel wants are contiguous, and a warp's stores of one column
+// are 128 contiguous bytes.
 template <int NMAX>
 __device__ __forceinline__ size_t slot_off(int half, int ch, int r) {
     return ((static_cast<size_t>(half) * (NMAX / 16) + ch) * BM + r) * 16;
 }
+__device__ __forceinline__ size_t slot_off_col(int col, int r) { return static_cast<size_t>(col) * BM + r; }
 __device__ __forceinline__ void slot_store16(float* dst, const float (&v)[16]) {
     float4* d = reinterpret_cast<float4*>(dst);
 #pragma unroll
     for (int q = 0; q < 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
+// va += the first 4*NQ columns of chunk ch, row r, of every contributor's
+// single-half slot, contributors in CTA order, 8/NQ contributors per round.
+template <int NQ, typename SlotOf>
+__device__ __forceinline__ void slot_sum_col(SlotOf slot_of, int c_first, int c_last, int ch, int r,
+                                             float (&va)[16]) {
+    constexpr int CB = 8 / NQ;
+    int c2 = c_first;
+    while (true) {
+        const float* src[CB];
+        int nb = 0;
+        for (; c2 <= c_last && nb < CB; ++c2) {
+            const float* sl = slot_of(c2);
+            if (sl) src[nb++] = sl;
+        }
+        if (nb == 0) break;
+        float x[CB][4 * NQ];
+#pragma unroll
+        for (int u = 0; u < CB; ++u)
+            if (u < nb) {
+#pragma unroll
+                for (int j = 0; j < 4 * NQ; ++j) x[u][j] = __ldcg(src[u] + slot_off_col(ch * 16 + j, r));
+            }
+#pragma unroll
+        for (int u = 0; u < CB; ++u)
+            if (u < nb) {
+#pragma unroll
+                for (int j = 0; j < 4 * NQ; ++j) va[j] += x[u][j];
+            }
+    }
+}
+
 // va (and vb, for GEMM1's second half) += the first 4*NQ values of every
 // contributor's slot of chunk ch, row r, contributors in CTA order.  The loads
 // of 8/NQ contributors (both halves) are issued before any addition, so the
@@ -445,6 +494,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
     using L = Layout<MODE, NMAX>;
     constexpr bool kStream = Cfg<MODE>::kStream;
+    constexpr int kSub = Cfg<MODE>::kSub;
     constexpr bool kG1 = Cfg<MODE>::kG1;
     constexpr int ST = L::STAGES;
 
@@ -491,6 +541,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int q_issued = 0;                       // k-steps whose loads were issued
     int npre = 0;                           // k-steps whose weight half was prefetched
     auto weight_loads = [&](const Work& w, int kt, uint32_t a, uint32_t b, uint32_t full) {
+        auto ld = [&](uint32_t dst, const CUtensorMap* m, int y, int z) { tma_load_3d(dst, m, full, 0, y, z); };
         const bool shared = p.offsets != nullptr && w.g == p.E;
         const int kx = kt * BK;
         if (MODE == G1_STREAM || MODE == G1_TILED) {
@@ -498,27 +549,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const CUtensorMap* wm = &maps.w_a;
             if (shared) { z = fl / p.I; fl -= z * p.I; wm = &maps.w_s; }
             const uint32_t dst = MODE == G1_STREAM ? a : b;
-            tma_load_3d(dst, wm, full, 0, packed_row(fl, kt, kt_h), z);
-            tma_load_3d(dst + TILE_BYTES, wm, full, 0, packed_row(p.I + fl, kt, kt_h), z);
+            ld(dst, wm, packed_row(fl, kt, kt_h), z);
+            ld(dst + TILE_BYTES, wm, packed_row(p.I + fl, kt, kt_h), z);
         } else if (MODE == G2_STREAM) {
             const int f0 = w.n * BM;
-            if (shared) {
-                const int z = kx / p.I;
-                tma_load_3d(a, &maps.w_s, full, 0, packed_row(f0, (kx - z * p.I) / BK, kt_i), z);
-            } else {
-                tma_load_3d(a, &maps.w_a, full, 0, packed_row(f0, kt, kt_i), w.g);
+#pragma unroll
+            for (int sb = 0; sb < kSub; ++sb) {
+                const int kb = kt * kSub + sb, kxb = kb * BK;
+                if (shared) {
+                    const int z = kxb / p.I;
+                    ld(a + sb * TILE_BYTES, &maps.w_s, packed_row(f0, (kxb - z * p.I) / BK, kt_i), z);
+                } else {
+                    ld(a + sb * TILE_BYTES, &maps.w_a, packed_row(f0, kb, kt_i), w.g);
+                }
             }
         } else if (MODE == LM_STREAM) {
-            tma_load_3d(a, &maps.w_a, full, 0, packed_row(w.n * BM, kt, kt_h), 0);
+#pragma unroll
+            for (int sb = 0; sb < kSub; ++sb)
+                ld(a + sb * TILE_BYTES, &maps.w_a, packed_row(w.n * BM, kt * kSub + sb, kt_h), 0);
         } else {   // G2_TILED
             const int n0 = w.n * p.bn;
             for (int j = 0; j < p.bn / BM; ++j) {
                 if (shared) {
                     const int z = kx / p.I;
-                    tma_load_3d(b + j * TILE_BYTES, &maps.w_s, full, 0,
-                                packed_row(n0 + j * BM, (kx - z * p.I) / BK, kt_i), z);
+                    ld(b + j * TILE_BYTES, &maps.w_s, packed_row(n0 + j * BM, (kx - z * p.I) / BK, kt_i), z);
                 } else {
-                    tma_load_3d(b + j * TILE_BYTES, &maps.w_a, full, 0, packed_row(n0 + j * BM, kt, kt_i), w.g);
+                    ld(b + j * TILE_BYTES, &maps.w_a, packed_row(n0 + j * BM, kt, kt_i), w.g);
                 }
             }
         }
@@ -526,7 +582,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     auto weight_bytes = [&]() -> uint32_t {
         if (MODE == G1_STREAM || MODE == G1_TILED) return 2 * TILE_BYTES;
         if (MODE == G2_TILED) return p.bn * BK * 2;
-        return TILE_BYTES;
+        return kSub * TILE_BYTES;
     };
     auto token_loads = [&](const Work& w, int kt, uint32_t a, uint32_t b, uint32_t full) -> uint32_t {
         const bool shared = p.offsets != nullptr && w.g == p.E;
@@ -534,8 +590,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int row0 = sched.row0[w.g];
         if (kStream) {
             const int nb = (sched.rows[w.g] + TOKBOX - 1) / TOKBOX;
-            mbar_expect_tx(full, nb * TOKBOX * BK * 2);
-            for (int j = 0; j < nb; ++j) tma_load_3d(b + j * TOKBOX * BK * 2, tm, full, kt * BK, row0 + j * TOKBOX, 0);
+            mbar_expect_tx(full, kSub * nb * TOKBOX * BK * 2);
+#pragma unroll
+            for (int sb = 0; sb < kSub; ++sb)
+                for (int j = 0; j < nb; ++j)
+                    tma_load_3d(b + sb * NMAX * BK * 2 + j * TOKBOX * BK * 2, tm, full, (kt * kSub + sb) * BK,
+                                row0 + j * TOKBOX, 0);
         } else {
             mbar_expect_tx(full, TILE_BYTES);
             tma_load_3d(a, tm, full, kt * BK, row0 + w.m0, 0);
@@ -545,7 +605,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (threadIdx.x == 0) {
         // Weight tiles do not depend on the previous kernel: start streaming
-        // the first stages now, while it drains.
+        // the first stages now, while it drains.  (Prefetching further
+        // k-steps into L2 as well measured slower: the extra requests delay
+        // the ones the pipeline waits for.)
         WorkIter<MODE> it;
         it.init(p, sched, c, nct);
         Work w;
@@ -642,15 +704,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 if (q == 0) tstamp(p, MODE, TS_FIRST_DATA);
                 tc_fence_after();
-                const uint32_t a = sbase + stage * L::STAGE;
-                const uint32_t b = a + L::A_BYTES;
+                const uint32_t a0 = sbase + stage * L::STAGE;
+                const uint32_t b0 = a0 + L::A_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk) {
-                    const uint32_t accum = (kt > w.k0 || kk > 0) ? 1u : 0u;
-                    const uint64_t bd = smem_desc_sw128(b + kk * 32);
-                    mma_bf16(d0, smem_desc_sw128(a + kk * 32), bd, idesc, accum);
-                    if (MODE == G1_STREAM)
-                        mma_bf16(d0 + 128, smem_desc_sw128(a + TILE_BYTES + kk * 32), bd, idesc, accum);
+                for (int sb = 0; sb < kSub; ++sb) {
+                    const uint32_t a = a0 + sb * TILE_BYTES, b = b0 + sb * NMAX * BK * 2;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint32_t accum = (kt > w.k0 || sb > 0 || kk > 0) ? 1u : 0u;
+                        const uint64_t bd = smem_desc_sw128(b + kk * 32);
+                        mma_bf16(d0, smem_desc_sw128(a + kk * 32), bd, idesc, accum);
+                        if (MODE == G1_STREAM)
+                            mma_bf16(d0 + 128, smem_desc_sw128(a + TILE_BYTES + kk * 32), bd, idesc, accum);
+                    }
                 }
                 mma_commit(smem_addr(&bar_empty[stage]));
             }
@@ -729,8 +795,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (kG1) tmem_ld16(tmem_at(128 + ch * 16), vb);
                     tmem_ld_wait();
                     if (!whole) {
-                        slot_store16(my_slot + slot_off<NMAX>(0, ch, r_in), va);
-                        if (kG1) slot_store16(my_slot + slot_off<NMAX>(1, ch, r_in), vb);
+                        if (kG1) {
+                            slot_store16(my_slot + slot_off<NMAX>(0, ch, r_in), va);
+                            slot_store16(my_slot + slot_off<NMAX>(1, ch, r_in), vb);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) my_slot[slot_off_col(ch * 16 + j, r_in)] = va[j];
+                        }
                         continue;
                     }
 #pragma unroll
@@ -866,9 +937,15 @@ __global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p)
 #pragma unroll
     for (int j = 0; j < 16; ++j) va[j] = vb[j] = 0.f;
     const int rc = rows - ch * 16;   // tokens of this chunk (only those are read)
-    if (rc <= 4) slot_sum<NMAX, 1, kG1>(slot_of, c_first, c_last, ch, r, va, vb);
-    else if (rc <= 8) slot_sum<NMAX, 2, kG1>(slot_of, c_first, c_last, ch, r, va, vb);
-    else slot_sum<NMAX, 4, kG1>(slot_of, c_first, c_last, ch, r, va, vb);
+    if (kG1) {
+        if (rc <= 4) slot_sum<NMAX, 1, true>(slot_of, c_first, c_last, ch, r, va, vb);
+        else if (rc <= 8) slot_sum<NMAX, 2, true>(slot_of, c_first, c_last, ch, r, va, vb);
+        else slot_sum<NMAX, 4, true>(slot_of, c_first, c_last, ch, r, va, vb);
+    } else {
+        if (rc <= 4) slot_sum_col<1>(slot_of, c_first, c_last, ch, r, va);
+        else if (rc <= 8) slot_sum_col<2>(slot_of, c_first, c_last, ch, r, va);
+        else slot_sum_col<4>(slot_of, c_first, c_last, ch, r, va);
+    }
     fin_stamp<MODE>(p, TS_FIRST_DATA);
     const bool shared = p.offsets != nullptr && g == p.E;
     const int f = n * BM + r;

@@ -122,6 +122,10 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // ------------------------------------------------------------ device side
 // Wait for the kernel this one depends on (no-op when launched without PDL).
+// Every kernel of this library calls grid_dep_launch only after its own
+// grid_dep_wait, so when kernel N starts, kernel N-2 has completed and its
+// writes are visible: a kernel may read what came from two or more launches
+// back before its own wait, and only what its direct predecessor writes after.
 __device__ __forceinline__ void grid_dep_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
