@@ -149,10 +149,11 @@ class ClockSampler:
 class Problem:
     """Device-resident weights and inputs of one workload (GPU-generated, seeded)."""
 
-    def __init__(self, shp: synth.MoEShape, n_sets: int, seed: int, device):
+    def __init__(self, shp: synth.MoEShape, n_sets: int, seed: int, device, fused_head: bool = False):
         import torch
         from speculative_decoding_verification_router_b200 import moespec as ms
         self.shp, self.ms, self.dev = shp, ms, device
+        self.fused_head = fused_head
         g = torch.Generator(device=device)
         g.manual_seed(seed)
 
@@ -176,7 +177,7 @@ class Problem:
         self.a = randn((T, H), 1.0, torch.float32)
         self.out = torch.empty((T, H), dtype=torch.float32, device=device)
         self.ws = ms.Workspace(ms.layer_workspace_size(T, H, E, I, S, k), device)
-        self.verify = shp.K > 0
+        self.verify = shp.K > 0 or shp.layers > 1   # the decode step always verifies (K = 0: greedy pick)
         if self.verify:
             B, K, V = shp.B, shp.K, shp.V
             self.lm = ms.pack_weights(randn((V, H), shp.weight_std, torch.bfloat16)) if shp.layers > 1 else None
@@ -186,6 +187,8 @@ class Problem:
                            for _ in range(self.n_logit_sets)]
             self.vws = ms.Workspace(ms.lib().spec_verify_workspace_size(B, K, V), device)
             self.lmws = ms.Workspace(ms.lib().lm_head_workspace_size(T, H, V), device) if self.lm is not None else None
+            self.fws = (ms.Workspace(ms.lib().spec_verify_lm_head_workspace_size(B, K, H, V), device)
+                        if self.lm is not None else None)
             self.h = [torch.empty((T, H), dtype=torch.float32, device=device) for _ in range(2)]
             self.xn = torch.empty((T, H), dtype=torch.bfloat16, device=device)
             am = torch.empty((B, K + 1), dtype=torch.int32, device=device)
@@ -219,8 +222,12 @@ class Problem:
             self.layer(l, cur, nxt)
             cur = nxt
         self.ms.rmsnorm(cur, out=self.xn)
-        self.ms.lm_head(self.xn, self.lm, ws=self.lmws, out=self.logits[0])
-        self.ms.verify_greedy(self.logits[0].view(s.B, s.K + 1, s.V), self.draft, ws=self.vws, out=self.vout)
+        if self.fused_head:
+            # vocab head with the argmax in its epilogue, then the prefix match
+            self.ms.verify_lm_head_greedy(self.xn, self.lm, self.draft, ws=self.fws, out=self.vout)
+        else:
+            self.ms.lm_head(self.xn, self.lm, ws=self.lmws, out=self.logits[0])
+            self.ms.verify_greedy(self.logits[0].view(s.B, s.K + 1, s.V), self.draft, ws=self.vws, out=self.vout)
 
     def units_per_step(self) -> int:
         return self.shp.T
@@ -265,7 +272,7 @@ def run_ours(args, rank, world, local):
 
     shp = WORKLOADS[args.workload]
     n_sets = args.sets or {"verify_b1": 4, "verify_b32": 4, "step12_b32": 12, "prefill": 1}[args.workload]
-    prob = Problem(shp, n_sets, seed=1234 + rank, device=device)
+    prob = Problem(shp, n_sets, seed=1234 + rank, device=device, fused_head=args.fused_head)
     stream = torch.cuda.Stream(device)
     torch.cuda.synchronize()
 
@@ -377,7 +384,9 @@ def run_ours(args, rank, world, local):
                    "parallelism": f"replicas{world}",
                    "l2": (f"rotating {n_sets} distinct weight sets "
                           f"({n_sets * (shp.E + shp.S) * EXPERT_BYTES(shp) / 1e9:.2f} GB) > 126 MB L2"),
-                   "graph": f"CUDA graph of {steps_per_graph} step(s), replayed {reps} times"},
+                   "graph": f"CUDA graph of {steps_per_graph} step(s), replayed {reps} times",
+                   **({"vocab_head": "fused (argmax in the GEMM epilogue)" if args.fused_head
+                       else "unfused (logits written, then verified)"} if shp.layers > 1 else {})},
         "roofline": roofline,
         "breakdown_us_per_step": {k: round(v, 2) for k, v in sorted(breakdown.items(), key=lambda kv: -kv[1])},
         "e2e": e2e,
@@ -534,6 +543,73 @@ def run_reference(args, rank, world):
     return line
 
 
+def run_k_sweep(args, rank, world, local):
+    """The 12-layer decode step at B = 32 for K = 0 (plain greedy decoding, one
+    token per step) and K = 1..3 drafts, each captured as one CUDA graph and
+    replayed.  Reports per K the step time, tau (tokens committed per sequence
+    per step, from the verification of drafts that match w.p. p_match), the
+    spec-step cost c(K) = t_step(K) / t_step(0) in plain-decoding steps, and
+    the speedup tau / c over plain greedy decoding."""
+    import dataclasses
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    base = synth.STEP_B32
+    sampler = ClockSampler(local)
+    sampler.start()
+    rows = []
+    for K in (0, 1, 2, 3):
+        shp = dataclasses.replace(base, name=f"{base.name}_K{K}", K=K)
+        prob = Problem(shp, 12, seed=1234 + rank, device=device, fused_head=args.fused_head)
+        stream = torch.cuda.Stream(device)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                prob.step(i)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            prob.step(0)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            graph.replay()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        t_ms = max_over_ranks(ev0.elapsed_time(ev1), world, device) / args.steps
+        n = prob.vout[2].cpu().numpy()
+        tau = float(n.mean())
+        rows.append({"K": K, "ms_per_step": round(t_ms, 5), "tau": round(tau, 4),
+                     "tau_closed_form": round(metrics.expected_tau_iid(shp.p_match, K), 4) if K else 1.0,
+                     "committed_tok_s": round(shp.B * tau / (t_ms / 1e3) * world, 1)})
+        del graph, prob
+        torch.cuda.empty_cache()
+    sampler.stop()
+    t0 = rows[0]["ms_per_step"]
+    for r in rows:
+        r["c"] = round(r["ms_per_step"] / t0, 4)
+        r["speedup"] = round(r["tau"] / r["c"], 4)
+    best = max(rows, key=lambda r: r["speedup"])
+    return {"metric": "speedup of the 12-layer speculative decode step over plain greedy decoding, K swept 0..3",
+            "value": rows[-1]["speedup"], "unit": "x (K=3)", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": base.name, "B": base.B, "layers": base.layers, "V": base.V,
+                       "p_match": base.p_match, "graph": "one CUDA graph per K, replayed",
+                       "vocab_head": "fused" if args.fused_head else "unfused",
+                       "l2": "12 distinct weight sets (5.5 GB) > 126 MB L2"},
+            "best_K": best["K"], "sweep": rows, "clocks": sampler.summary()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -544,6 +620,11 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sets", type=int, default=0, help="distinct weight sets rotated across steps (0 = workload default)")
+    ap.add_argument("--k-sweep", action="store_true",
+                    help="12-layer step at B=32 for K = 0..3: step time, tau, spec-step cost and speedup")
+    ap.add_argument("--fused-head", action="store_true",
+                    help="12-layer step: argmax in the vocab head's epilogue (spec_verify_lm_head_greedy) "
+                         "instead of writing the logits and verifying them in a separate kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -553,7 +634,7 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
         return
-    result = run_ours(args, rank, world, local)
+    result = run_k_sweep(args, rank, world, local) if args.k_sweep else run_ours(args, rank, world, local)
     if rank == 0:
         print(json.dumps(result), flush=True)
 

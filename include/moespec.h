@@ -36,7 +36,7 @@
  *    a kernel) are recorded in a status word inside the caller's workspace
  *    and read with ms_device_status(); the kernel then skips the affected
  *    work instead of trapping.
- *  - Sizes: 1 <= k <= E <= 256; H % 128 == 0; I % 128 == 0; 1 <= K <= 8.
+ *  - Sizes: 1 <= k <= E <= 256; H % 128 == 0; I % 128 == 0; 0 <= K <= 8 (K = 0: plain greedy).
  */
 #ifndef MOESPEC_H
 #define MOESPEC_H
@@ -165,12 +165,33 @@ MS_API ms_status lm_head_logits(const void* xhat, const void* w_lm, int T, int H
  * n = longest m <= K with draft[b,i] == argmax[b,i] for all i < m;
  * committed[b,:] = draft[b,0..n-1], argmax[b,n], then -1 padding;
  * n_committed[b] = n + 1, always in 1..K+1.
+ * K = 0 (no drafts; draft may be NULL) is plain greedy decoding: one row per
+ * sequence, committed[b,0] = its argmax, n_committed[b] = 1.
  * argmax, committed: [B,K+1] int32.  n_committed: [B] int32.
  * Scratch: spec_verify_workspace_size(B,K,V) bytes (partial maxima). */
 MS_API size_t spec_verify_workspace_size(int B, int K, int V);
 MS_API ms_status spec_verify_greedy(const void* logits, ms_dtype logits_dtype, const int32_t* draft,
                              int B, int K, int V, int32_t* argmax, int32_t* committed,
                              int32_t* n_committed, void* ws, size_t ws_bytes, void* stream);
+
+/* a5 + a6 fused: the vocab head with the verification's argmax in its
+ * epilogue, then the prefix match -- the logits are never written.
+ * xhat: [B*(K+1),H] bf16, the final hidden states of the verify rows (row
+ * b*(K+1)+j scores the token after position j of sequence b).
+ * w_lm: [V,H] bf16 packed by moe_pack_weights (n=1, rows=V, cols=H).
+ * The argmax of row t is taken over the bf16 rounding of the fp32 logits
+ * sum_h xhat[t,h] w_lm[v,h], lowest index among equal values (-0 equals +0),
+ * i.e. over exactly the logits lm_head_logits writes; argmax, committed and
+ * n_committed then follow spec_verify_greedy (K = 0 included).  K <= 8, H % 128 == 0,
+ * V % 128 == 0.  NaN logits are not supported.  Each quarter of a
+ * 128-row vocabulary tile stores its per-row maximum as a 64-bit key (value
+ * order << 32 | ~index) in its own slot, and the verify kernel takes each
+ * row's largest key: exact, no atomics, deterministic.
+ * Scratch: spec_verify_lm_head_workspace_size(B,K,H,V) bytes. */
+MS_API size_t spec_verify_lm_head_workspace_size(int B, int K, int H, int V);
+MS_API ms_status spec_verify_lm_head_greedy(const void* xhat, const void* w_lm, const int32_t* draft, int B,
+                                            int K, int H, int V, int32_t* argmax, int32_t* committed,
+                                            int32_t* n_committed, void* ws, size_t ws_bytes, void* stream);
 
 /* Allocation-free variant of spec_verify_greedy.  The pages have no
  * counterpart: this exists for callers that cannot allocate device memory,

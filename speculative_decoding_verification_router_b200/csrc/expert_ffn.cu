@@ -71,6 +71,7 @@ struct Params {
     int y_bf16;
     float* y_sh;                   // [T][H]
     __nv_bfloat16* logits;         // [T][V]
+    unsigned long long* amax_key;  // vocab head, fused argmax: [T][4 V/128] keys instead of logits
     float* partials;               // 2 partial-sum slots per CTA (streaming)
     int nct;                       // grid size of the streaming GEMM (for the finish kernel)
     int32_t* status;
@@ -390,6 +391,32 @@ __device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, uint64_t
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+// Order-preserving 16-bit key of the bf16 rounding of v: a larger value has a
+// larger key, and -0 is taken as +0 (they compare equal).  NaN is not ordered.
+__device__ __forceinline__ uint32_t bf16_order_key(float v) {
+    uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    if (b == 0x8000u) b = 0;
+    return (b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u);
+}
+
+// Fused argmax of the vocab head: the largest bf16 logit of token t over the
+// 32 vocabulary rows of this warp (quarter `quad` of tile `tile`), lowest row
+// on ties, by one warp max over (value key << 16 | 65535 - row), stored as a
+// 64-bit key (value key << 32 | ~vocabulary index) in slot (t, 4 tile + quad)
+// of a [T][4 V/128] table.  Every slot is written exactly once; the verify
+// kernel takes the max over a row's slots: largest value, then lowest index.
+// Called by all 32 lanes of a warp with the same token.
+__device__ __forceinline__ void argmax_store(unsigned long long* keys, int ld, int t, float v, int row_in_tile,
+                                             int tile, int quad, int lane) {
+    uint32_t k32 = (bf16_order_key(v) << 16) | (0xFFFFu - static_cast<uint32_t>(row_in_tile));
+    k32 = __reduce_max_sync(0xffffffffu, k32);
+    if (lane == 0) {
+        const uint32_t idx = static_cast<uint32_t>(tile) * BM + (0xFFFFu - (k32 & 0xFFFFu));
+        keys[static_cast<size_t>(t) * ld + tile * 4 + quad] =
+            (static_cast<unsigned long long>(k32 >> 16) << 32) | (0xFFFFFFFFu - idx);
+    }
+}
 
 // Partial-sum slot of a split tile.  GEMM1 (gate and up halves):
 // [half][chunk][row][16], so a thread's 16 values of one chunk are 64
@@ -804,6 +831,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         }
                         continue;
                     }
+                    if (MODE == LM_STREAM && p.amax_key) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (ch * 16 + j < rows)
+                                argmax_store(p.amax_key, 4 * (p.V / BM), ch * 16 + j, va[j], r_in, w.n, q4, lane);
+                        continue;
+                    }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int t = ch * 16 + j;
@@ -947,6 +981,13 @@ __global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p)
         else slot_sum_col<4>(slot_of, c_first, c_last, ch, r, va);
     }
     fin_stamp<MODE>(p, TS_FIRST_DATA);
+    if (MODE == LM_STREAM && p.amax_key) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (ch * 16 + j < rows) argmax_store(p.amax_key, 4 * (p.V / BM), ch * 16 + j, va[j], r, n, r >> 5, r & 31);
+        fin_stamp<MODE>(p, TS_EXIT);
+        return;
+    }
     const bool shared = p.offsets != nullptr && g == p.E;
     const int f = n * BM + r;
 #pragma unroll
@@ -1209,8 +1250,10 @@ static LmWs lm_ws_layout(void* base, int H, int V) {
 
 size_t lm_ws_bytes(int H, int V) { return lm_ws_layout(nullptr, H, V).bytes; }
 
+// keys != nullptr: fused argmax -- no logits; keys [T][4 V/128] receives the
+// per-tile-quarter argmax keys of every row (see argmax_store).
 ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* logits, void* ws,
-                    cudaStream_t s) {
+                    cudaStream_t s, unsigned long long* keys = nullptr) {
     LmWs w = lm_ws_layout(ws, H, V);
     for (int t0 = 0; t0 < T; t0 += BM) {
         const int tc = T - t0 < BM ? T - t0 : BM;
@@ -1227,7 +1270,8 @@ ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* l
         prm.T = tc; prm.H = H; prm.E = 1; prm.I = BM; prm.S = 0; prm.k = 1; prm.V = V;
         prm.bn = 128;
         prm.offsets = nullptr;
-        prm.logits = reinterpret_cast<__nv_bfloat16*>(logits) + static_cast<size_t>(t0) * V;
+        prm.logits = keys ? nullptr : reinterpret_cast<__nv_bfloat16*>(logits) + static_cast<size_t>(t0) * V;
+        prm.amax_key = keys ? keys + static_cast<size_t>(t0) * 4 * (V / BM) : nullptr;
         prm.partials = w.partials;
         prm.status = w.status;
         prm.wait_limit_ns = wait_limit_ns();
@@ -1271,6 +1315,41 @@ extern "C" ms_status moe_expert_ffn(const void* xhat, const int32_t* expert_offs
     }
     return ms::ffn_launch(xhat, expert_offsets, perm_token, w_gate_up, w_down, ws_gate_up, ws_down, T, H, E,
                           I, S, k, y_perm, y_perm_dtype, y_shared, ws, static_cast<cudaStream_t>(stream));
+}
+
+namespace ms {
+ms_status verify_keys_launch(const unsigned long long*, int, int, int, const int32_t*, int32_t*, int32_t*,
+                             int32_t*, cudaStream_t);
+}
+
+extern "C" size_t spec_verify_lm_head_workspace_size(int B, int K, int H, int V) {
+    if (B <= 0 || K < 0 || H <= 0 || V <= 0) return 0;
+    return ms::lm_ws_bytes(H, V) + ms::align_up(static_cast<size_t>(B) * (K + 1) * 4 * (V / 128) * 8, 1024);
+}
+
+extern "C" ms_status spec_verify_lm_head_greedy(const void* xhat, const void* w_lm, const int32_t* draft, int B,
+                                                int K, int H, int V, int32_t* argmax, int32_t* committed,
+                                                int32_t* n_committed, void* ws, size_t ws_bytes, void* stream) {
+    if (!xhat || !w_lm || (K > 0 && !draft) || !argmax || !committed || !n_committed) return MS_ERR_INVALID_ARG;
+    if (B <= 0 || K < 0 || H <= 0 || V <= 0) return MS_ERR_INVALID_ARG;
+    if (K > 8 || H % 128 != 0 || V % 128 != 0 || V > (1 << 30)) return MS_ERR_UNSUPPORTED;
+    if (static_cast<long>(B) * (K + 1) > (1L << 24)) return MS_ERR_UNSUPPORTED;
+    if (!ms::aligned16(xhat) || !ms::aligned16(w_lm)) return MS_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < spec_verify_lm_head_workspace_size(B, K, H, V)) return MS_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 1023u) return MS_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int T = B * (K + 1);
+    const size_t lm_bytes = ms::lm_ws_bytes(H, V);
+    auto* keys = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + lm_bytes);
+    // the status word starts at zero; every key slot is written by the head
+    cudaError_t ce = cudaMemsetAsync(ws, 0, sizeof(int32_t), s);
+    if (ce != cudaSuccess) {
+        ms::set_cuda_error(ce);
+        return MS_ERR_CUDA;
+    }
+    ms_status st = ms::lm_launch(xhat, w_lm, T, H, V, nullptr, ws, s, keys);
+    if (st != MS_OK) return st;
+    return ms::verify_keys_launch(keys, 4 * (V / 128), B, K, draft, argmax, committed, n_committed, s);
 }
 
 extern "C" size_t lm_head_workspace_size(int T, int H, int V) {

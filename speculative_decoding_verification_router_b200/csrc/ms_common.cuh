@@ -31,6 +31,7 @@ enum KernelId : int {
     K_VERIFY_PARTIAL,
     K_VERIFY_FINAL,
     K_VERIFY_CLUSTER,
+    K_VERIFY_KEYS,
     K_WAIT_PROBE,
     K_PACK,
     K_COUNT

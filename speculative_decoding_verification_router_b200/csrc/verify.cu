@@ -123,6 +123,79 @@ __global__ void __launch_bounds__(128) verify_final_kernel(const float* __restri
     }
 }
 
+// Greedy verification from the fused vocab head's argmax keys: keys is a
+// [B(K+1)][ld] table of 64-bit keys (order key of a bf16 value << 32 | ~index);
+// the largest key of a row gives its largest value and, among equal values,
+// the lowest index.  One 1024-thread block per sequence: every thread takes a
+// strided share of all K+1 rows at once (its loads all in flight together),
+// then warp and block maxima.
+constexpr int VK_THREADS = 1024;
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = w > v ? w : v;
+    }
+    return v;
+}
+
+__global__ void __launch_bounds__(VK_THREADS) verify_keys_kernel(const unsigned long long* __restrict__ keys,
+                                                                 int ld, int K, const int32_t* __restrict__ draft,
+                                                                 int32_t* __restrict__ argmax,
+                                                                 int32_t* __restrict__ committed,
+                                                                 int32_t* __restrict__ n_committed) {
+    __shared__ unsigned long long red[VK_THREADS / 32][kMaxK + 1];
+    grid_dep_wait();
+    grid_dep_launch();
+    const int b = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned long long m[kMaxK + 1];
+#pragma unroll
+    for (int j = 0; j <= kMaxK; ++j) m[j] = 0;
+#pragma unroll 4
+    for (int q = threadIdx.x; q < ld; q += VK_THREADS) {
+#pragma unroll
+        for (int j = 0; j <= kMaxK; ++j)
+            if (j <= K) {
+                const unsigned long long v = __ldcg(keys + (static_cast<size_t>(b) * (K + 1) + j) * ld + q);
+                m[j] = v > m[j] ? v : m[j];
+            }
+    }
+#pragma unroll
+    for (int j = 0; j <= kMaxK; ++j)
+        if (j <= K) {
+            const unsigned long long v = warp_max_u64(m[j]);
+            if (lane == 0) red[warp][j] = v;
+        }
+    __syncthreads();
+    if (threadIdx.x != 0) return;
+    int g[kMaxK + 1];
+#pragma unroll
+    for (int j = 0; j <= kMaxK; ++j)
+        if (j <= K) {
+            unsigned long long v = 0;
+            for (int w = 0; w < VK_THREADS / 32; ++w) v = red[w][j] > v ? red[w][j] : v;
+            g[j] = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(v & 0xFFFFFFFFull));
+        }
+    int n = 0;
+    while (n < K && __ldg(draft + static_cast<size_t>(b) * K + n) == g[n]) ++n;
+    int32_t* am = argmax + static_cast<size_t>(b) * (K + 1);
+    int32_t* cm = committed + static_cast<size_t>(b) * (K + 1);
+    for (int j = 0; j <= K; ++j) {
+        am[j] = g[j];
+        cm[j] = j < n ? g[j] : (j == n ? g[n] : -1);
+    }
+    n_committed[b] = n + 1;
+}
+
+ms_status verify_keys_launch(const unsigned long long* keys, int ld, int B, int K, const int32_t* draft,
+                             int32_t* argmax, int32_t* committed, int32_t* n_committed, cudaStream_t s) {
+    if (K < 0 || K > kMaxK) return MS_ERR_UNSUPPORTED;
+    return launch(K_VERIFY_KEYS, verify_keys_kernel, dim3(B), dim3(VK_THREADS), 0, s, keys, ld, K, draft, argmax,
+                  committed, n_committed);
+}
+
 // Single-kernel verification: one thread-block cluster per sequence, CTA r of
 // the cluster scans chunk r % P of row r / P with 16-byte loads (several in
 // flight per thread), reduces (max, lowest index) in the block and stores the
@@ -372,8 +445,8 @@ extern "C" ms_status spec_verify_greedy_noalloc(const void* logits, ms_dtype log
                                                 const int32_t* draft, int B, int K, int V,
                                                 int32_t* argmax, int32_t* committed,
                                                 int32_t* n_committed, void* stream) {
-    if (!logits || !draft || !argmax || !committed || !n_committed) return MS_ERR_INVALID_ARG;
-    if (B <= 0 || V <= 0 || K < 1) return MS_ERR_INVALID_ARG;
+    if (!logits || (K > 0 && !draft) || !argmax || !committed || !n_committed) return MS_ERR_INVALID_ARG;
+    if (B <= 0 || V <= 0 || K < 0) return MS_ERR_INVALID_ARG;
     if (logits_dtype != MS_F32 && logits_dtype != MS_BF16) return MS_ERR_INVALID_ARG;
     if (K > ms::kMaxK) return MS_ERR_UNSUPPORTED;
     if (static_cast<long>(B) * (K + 1) * V > (1L << 40)) return MS_ERR_UNSUPPORTED;
@@ -387,7 +460,7 @@ extern "C" ms_status spec_verify_greedy_noalloc(const void* logits, ms_dtype log
 }
 
 extern "C" size_t spec_verify_workspace_size(int B, int K, int V) {
-    if (B <= 0 || K < 1 || V <= 0) return 0;
+    if (B <= 0 || K < 0 || V <= 0) return 0;
     return ms::verify_ws_bytes(B, K, V);
 }
 
@@ -396,8 +469,8 @@ extern "C" ms_status spec_verify_greedy(const void* logits, ms_dtype logits_dtyp
                                         int32_t* argmax, int32_t* committed,
                                         int32_t* n_committed, void* ws, size_t ws_bytes,
                                         void* stream) {
-    if (!logits || !draft || !argmax || !committed || !n_committed) return MS_ERR_INVALID_ARG;
-    if (B <= 0 || V <= 0 || K < 1) return MS_ERR_INVALID_ARG;
+    if (!logits || (K > 0 && !draft) || !argmax || !committed || !n_committed) return MS_ERR_INVALID_ARG;
+    if (B <= 0 || V <= 0 || K < 0) return MS_ERR_INVALID_ARG;
     if (logits_dtype != MS_F32 && logits_dtype != MS_BF16) return MS_ERR_INVALID_ARG;
     if (K > ms::kMaxK) return MS_ERR_UNSUPPORTED;
     if (static_cast<long>(B) * (K + 1) * V > (1L << 40)) return MS_ERR_UNSUPPORTED;

@@ -48,6 +48,8 @@ def _load():
         "lm_head_logits": (I, [P, P, I, I, I, P, P, Z, P]),
         "spec_verify_workspace_size": (Z, [I, I, I]),
         "spec_verify_greedy": (I, [P, I, P, I, I, I, P, P, P, P, Z, P]),
+        "spec_verify_lm_head_workspace_size": (Z, [I, I, I, I]),
+        "spec_verify_lm_head_greedy": (I, [P, P, P, I, I, I, I, P, P, P, P, Z, P]),
         "moe_layer_workspace_size": (Z, [I, I, I, I, I, I]),
         "moe_layer_forward": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, Z, P]),
         "ms_device_status": (I, [P, P]),
@@ -245,6 +247,27 @@ def verify_greedy(logits, draft, ws: Optional[Workspace] = None, out=None, strea
     w = _ws(ws, _lib.spec_verify_workspace_size(B, K, V), dev)
     _check(_lib.spec_verify_greedy(_p(logits), dt, _p(draft), B, K, V, _p(am), _p(cm), _p(n), w.c(), w.nbytes,
                                    _stream(stream)), "spec_verify_greedy")
+    return am, cm, n
+
+
+def verify_lm_head_greedy(xhat, w_lm, draft, ws: Optional[Workspace] = None, out=None, stream=None):
+    """Vocab head with the verification's argmax fused into its epilogue, then
+    the prefix match.  xhat [B*(K+1), H] bf16, w_lm packed [V, H] bf16, draft [B, K] int32."""
+    _dev(xhat, torch.bfloat16, "xhat")
+    _dev(w_lm, torch.bfloat16, "w_lm")
+    _dev(draft, torch.int32, "draft")
+    B, K = draft.shape
+    T, H = xhat.shape
+    V = w_lm.shape[0]
+    if T != B * (K + 1):
+        raise ValueError(f"xhat has {T} rows, expected B*(K+1) = {B * (K + 1)}")
+    dev = xhat.device
+    am, cm, n = out if out is not None else (torch.empty((B, K + 1), dtype=torch.int32, device=dev),
+                                             torch.empty((B, K + 1), dtype=torch.int32, device=dev),
+                                             torch.empty(B, dtype=torch.int32, device=dev))
+    w = _ws(ws, _lib.spec_verify_lm_head_workspace_size(B, K, H, V), dev)
+    _check(_lib.spec_verify_lm_head_greedy(_p(xhat), _p(w_lm), _p(draft), B, K, H, V, _p(am), _p(cm), _p(n),
+                                           w.c(), w.nbytes, _stream(stream)), "spec_verify_lm_head_greedy")
     return am, cm, n
 
 

@@ -52,6 +52,18 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.spec_verify_greedy(fake, 1, fake, 2, 3, 100, fake, fake, fake, None, 0, None) == -3  # no ws
     assert lib.spec_verify_greedy(fake, 1, fake, 2, 9, 100, fake, fake, fake, fake, 1 << 20, None) == -2  # K > 8
     assert lib.spec_verify_greedy(fake, 7, fake, 2, 3, 100, fake, fake, fake, fake, 1 << 20, None) == -1  # dtype
+    Z = ctypes.c_size_t
+    lib.spec_verify_lm_head_greedy.restype = I
+    lib.spec_verify_lm_head_greedy.argtypes = [P, P, P, I, I, I, I, P, P, P, P, Z, P]
+    lib.spec_verify_lm_head_workspace_size.restype = Z
+    lib.spec_verify_lm_head_workspace_size.argtypes = [I] * 4
+    fused = lib.spec_verify_lm_head_greedy
+    assert fused(None, fake, fake, 2, 3, 256, 1024, fake, fake, fake, fake, 1 << 30, None) == -1   # null xhat
+    assert fused(fake, fake, fake, 2, 9, 256, 1024, fake, fake, fake, fake, 1 << 30, None) == -2   # K > 8
+    assert fused(fake, fake, fake, 2, 3, 256, 1000, fake, fake, fake, fake, 1 << 30, None) == -2   # V % 128
+    assert fused(fake, fake, fake, 2, 3, 256, 1024, fake, fake, fake, None, 0, None) == -3         # no ws
+    assert lib.spec_verify_lm_head_workspace_size(32, 3, 1280, 129280) > 32 * 4 * 8
+    assert lib.spec_verify_lm_head_workspace_size(0, 3, 1280, 129280) == 0
     lib.moe_expert_ffn_workspace_size.restype = ctypes.c_size_t
     lib.moe_expert_ffn_workspace_size.argtypes = [I] * 6
     assert lib.moe_expert_ffn_workspace_size(4, 1280, 64, 896, 2, 6) > 0

@@ -53,7 +53,7 @@ def test_verify_ragged_vocab(ms, V, dtype):
     _check(ms, lg, d)
 
 
-@pytest.mark.parametrize("K", [1, 2, 8])
+@pytest.mark.parametrize("K", [0, 1, 2, 8])   # K = 0: plain greedy decoding
 def test_verify_depths(ms, K):
     shp = synth.MoEShape("depth", B=6, K=K, H=128, E=2, I=128, k=1, S=0, V=5000, router_std=1.0, p_match=0.8)
     lg, d = verify_inputs(shp, seed=3, dtype="bf16")

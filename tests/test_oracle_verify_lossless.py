@@ -94,6 +94,16 @@ def test_verify_invariants_random():
             np.testing.assert_array_equal(cm[b, : m + 1], am_true[b, : m + 1])
 
 
+def test_verify_without_drafts_is_greedy_decoding():
+    # K = 0: one row per sequence, its argmax committed, one token per step
+    g = np.random.default_rng(6)
+    lg = g.standard_normal((5, 1, 300)).astype(np.float32)
+    am, cm, n = oracle.verify_greedy(lg, np.zeros((5, 0), np.int32))
+    np.testing.assert_array_equal(am[:, 0], np.argmax(lg[:, 0], axis=1))
+    np.testing.assert_array_equal(cm, am)
+    assert np.all(n == 1)
+
+
 def test_mean_tau_matches_closed_form():
     # drafts match iid with p_eff = p + (1-p)/V; E[tau] = sum_{i<=K} p_eff^i
     shp = synth.TINY
