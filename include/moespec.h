@@ -183,10 +183,10 @@ MS_API ms_status spec_verify_greedy(const void* logits, ms_dtype logits_dtype, c
  * sum_h xhat[t,h] w_lm[v,h], lowest index among equal values (-0 equals +0),
  * i.e. over exactly the logits lm_head_logits writes; argmax, committed and
  * n_committed then follow spec_verify_greedy (K = 0 included).  K <= 8, H % 128 == 0,
- * V % 128 == 0.  NaN logits are not supported.  Each quarter of a
- * 128-row vocabulary tile stores its per-row maximum as a 64-bit key (value
- * order << 32 | ~index) in its own slot, and the verify kernel takes each
- * row's largest key: exact, no atomics, deterministic.
+ * V % 128 == 0.  NaN logits are not supported.  Each 16-row vocabulary
+ * chunk stores every row's maximum as a 64-bit key (value order << 32 |
+ * ~index) in its own slot, and the verify kernel takes each row's largest
+ * key: exact, no atomics, deterministic.
  * Scratch: spec_verify_lm_head_workspace_size(B,K,H,V) bytes. */
 MS_API size_t spec_verify_lm_head_workspace_size(int B, int K, int H, int V);
 MS_API ms_status spec_verify_lm_head_greedy(const void* xhat, const void* w_lm, const int32_t* draft, int B,

@@ -71,7 +71,7 @@ struct Params {
     int y_bf16;
     float* y_sh;                   // [T][H]
     __nv_bfloat16* logits;         // [T][V]
-    unsigned long long* amax_key;  // vocab head, fused argmax: [T][4 V/128] keys instead of logits
+    unsigned long long* amax_key;  // vocab head, fused argmax: [T][V/16] keys instead of logits (NMAX 128)
     float* partials;               // 2 partial-sum slots per CTA (streaming)
     int nct;                       // grid size of the streaming GEMM (for the finish kernel)
     int32_t* status;
@@ -400,22 +400,25 @@ __device__ __forceinline__ uint32_t bf16_order_key(float v) {
     return (b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u);
 }
 
-// Fused argmax of the vocab head: the largest bf16 logit of token t over the
-// 32 vocabulary rows of this warp (quarter `quad` of tile `tile`), lowest row
-// on ties, by one warp max over (value key << 16 | 65535 - row), stored as a
-// 64-bit key (value key << 32 | ~vocabulary index) in slot (t, 4 tile + quad)
-// of a [T][4 V/128] table.  Every slot is written exactly once; the verify
-// kernel takes the max over a row's slots: largest value, then lowest index.
-// Called by all 32 lanes of a warp with the same token.
-__device__ __forceinline__ void argmax_store(unsigned long long* keys, int ld, int t, float v, int row_in_tile,
-                                             int tile, int quad, int lane) {
-    uint32_t k32 = (bf16_order_key(v) << 16) | (0xFFFFu - static_cast<uint32_t>(row_in_tile));
-    k32 = __reduce_max_sync(0xffffffffu, k32);
-    if (lane == 0) {
-        const uint32_t idx = static_cast<uint32_t>(tile) * BM + (0xFFFFu - (k32 & 0xFFFFu));
-        keys[static_cast<size_t>(t) * ld + tile * 4 + quad] =
-            (static_cast<unsigned long long>(k32 >> 16) << 32) | (0xFFFFFFFFu - idx);
+// Fused argmax of the vocab head.  In this mode the accumulator is token-major
+// (TMEM lane = token, column = vocabulary row of the tile), so a thread scans
+// the 16 logits of one 16-row vocabulary chunk of its own token: each is
+// rounded to bf16 and mapped to (order key << 16 | 65535 - column); the
+// largest such word is the chunk's largest value at its lowest index.  It is
+// stored as a 64-bit key (value key << 32 | ~vocabulary index) in slot
+// (t, chunk) of a [T][V/16] table, every slot written exactly once; the
+// verify kernel takes the max over a row's slots: largest value, then lowest
+// index.
+__device__ __forceinline__ void argmax_chunk_store(unsigned long long* keys, int ld, int t, const float (&v)[16],
+                                                   int chunk) {
+    uint32_t best = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const uint32_t k = (bf16_order_key(v[j]) << 16) | (0xFFFFu - static_cast<uint32_t>(j));
+        best = k > best ? k : best;
     }
+    const uint32_t idx = static_cast<uint32_t>(chunk) * 16 + (0xFFFFu - (best & 0xFFFFu));
+    keys[static_cast<size_t>(t) * ld + chunk] = (static_cast<unsigned long long>(best >> 16) << 32) | (0xFFFFFFFFu - idx);
 }
 
 // Partial-sum slot of a split tile.  GEMM1 (gate and up halves):
@@ -522,6 +525,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     using L = Layout<MODE, NMAX>;
     constexpr bool kStream = Cfg<MODE>::kStream;
     constexpr int kSub = Cfg<MODE>::kSub;
+    // vocab head with the fused argmax: tokens are the MMA's M operand, vocabulary rows its N
+    const bool tokM = MODE == LM_STREAM && p.amax_key != nullptr;
     constexpr bool kG1 = Cfg<MODE>::kG1;
     constexpr int ST = L::STAGES;
 
@@ -616,7 +621,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const CUtensorMap* tm = shared ? &maps.tok_s : &maps.tok_r;
         const int row0 = sched.row0[w.g];
         if (kStream) {
-            const int nb = (sched.rows[w.g] + TOKBOX - 1) / TOKBOX;
+            // token-major argmax mode: the tokens are the M = 128 operand, all 128 rows
+            const int nb = tokM ? BM / TOKBOX : (sched.rows[w.g] + TOKBOX - 1) / TOKBOX;
             mbar_expect_tx(full, kSub * nb * TOKBOX * BK * 2);
 #pragma unroll
             for (int sb = 0; sb < kSub; ++sb)
@@ -719,7 +725,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!mbar_wait(smem_addr(&bar_tempty[acc]), acc_phase ^ 1u, lim, &abort_sh)) { ok = false; break; }
             tc_fence_after();
             uint32_t n_mma;
-            if (kStream) n_mma = static_cast<uint32_t>((sched.rows[w.g] + 15) / 16 * 16);
+            if (tokM) n_mma = BM;
+            else if (kStream) n_mma = static_cast<uint32_t>((sched.rows[w.g] + 15) / 16 * 16);
             else n_mma = MODE == G1_TILED ? 256u : static_cast<uint32_t>(p.bn);
             const uint32_t idesc = idesc_bf16_f32(BM, n_mma);
             const uint32_t d0 = tmem_base + acc * 256;
@@ -740,6 +747,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint32_t accum = (kt > w.k0 || sb > 0 || kk > 0) ? 1u : 0u;
                         const uint64_t bd = smem_desc_sw128(b + kk * 32);
+                        if (MODE == LM_STREAM && tokM) {   // D[token][vocab row] = x . w
+                            mma_bf16(d0, bd, smem_desc_sw128(a + kk * 32), idesc, accum);
+                            continue;
+                        }
                         mma_bf16(d0, smem_desc_sw128(a + kk * 32), bd, idesc, accum);
                         if (MODE == G1_STREAM)
                             mma_bf16(d0 + 128, smem_desc_sw128(a + TILE_BYTES + kk * 32), bd, idesc, accum);
@@ -809,7 +820,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (kStream) {
                 const int slot_floats = BM * NMAX * (kG1 ? 2 : 1);
                 const int f = w.n * BM + r_in;          // output feature of this thread
-                const int nch = (rows + 15) / 16;
+                const int nch = tokM ? BM / 16 : (rows + 15) / 16;
                 const bool whole = w.k0 == 0 && w.k1 == w.kt;
                 float* my_slot = nullptr;
                 if (!whole) {
@@ -822,8 +833,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (kG1) tmem_ld16(tmem_at(128 + ch * 16), vb);
                     tmem_ld_wait();
                     if (!whole) {
-                        if (kG1) {
+                        if (kG1 || tokM) {   // token-major: [chunk][token][16 vocabulary rows]
                             slot_store16(my_slot + slot_off<NMAX>(0, ch, r_in), va);
+                            if (tokM) continue;
                             slot_store16(my_slot + slot_off<NMAX>(1, ch, r_in), vb);
                         } else {
 #pragma unroll
@@ -831,11 +843,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         }
                         continue;
                     }
-                    if (MODE == LM_STREAM && p.amax_key) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            if (ch * 16 + j < rows)
-                                argmax_store(p.amax_key, 4 * (p.V / BM), ch * 16 + j, va[j], r_in, w.n, q4, lane);
+                    if (tokM) {
+                        if (r_in < rows) argmax_chunk_store(p.amax_key, p.V / 16, r_in, va, w.n * (BM / 16) + ch);
                         continue;
                     }
 #pragma unroll
@@ -958,7 +967,7 @@ __global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p)
     if (c_first == c_last) return;   // one CTA did the whole tile and stored it
     const int rows = sched.rows[g], row0 = sched.row0[g];
     const int ch = blockIdx.y;
-    if (ch * 16 >= rows) return;
+    if (!(MODE == LM_STREAM && p.amax_key) && ch * 16 >= rows) return;   // (argmax mode: ch = vocabulary rows)
     constexpr bool kG1 = Cfg<MODE>::kG1;
     const int slot_floats = BM * NMAX * (kG1 ? 2 : 1);
     const int r = threadIdx.x;
@@ -970,6 +979,15 @@ __global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p)
     float va[16], vb[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) va[j] = vb[j] = 0.f;
+    if (MODE == LM_STREAM && p.amax_key) {
+        // token-major partials: thread = token, chunk ch = 16 vocabulary rows
+        if (r < rows) {
+            slot_sum<NMAX, 4, false>(slot_of, c_first, c_last, ch, r, va, vb);
+            argmax_chunk_store(p.amax_key, p.V / 16, r, va, n * (BM / 16) + ch);
+        }
+        fin_stamp<MODE>(p, TS_EXIT);
+        return;
+    }
     const int rc = rows - ch * 16;   // tokens of this chunk (only those are read)
     if (kG1) {
         if (rc <= 4) slot_sum<NMAX, 1, true>(slot_of, c_first, c_last, ch, r, va, vb);
@@ -981,13 +999,6 @@ __global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p)
         else slot_sum_col<4>(slot_of, c_first, c_last, ch, r, va);
     }
     fin_stamp<MODE>(p, TS_FIRST_DATA);
-    if (MODE == LM_STREAM && p.amax_key) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (ch * 16 + j < rows) argmax_store(p.amax_key, 4 * (p.V / BM), ch * 16 + j, va[j], r, n, r >> 5, r & 31);
-        fin_stamp<MODE>(p, TS_EXIT);
-        return;
-    }
     const bool shared = p.offsets != nullptr && g == p.E;
     const int f = n * BM + r;
 #pragma unroll
@@ -1250,8 +1261,8 @@ static LmWs lm_ws_layout(void* base, int H, int V) {
 
 size_t lm_ws_bytes(int H, int V) { return lm_ws_layout(nullptr, H, V).bytes; }
 
-// keys != nullptr: fused argmax -- no logits; keys [T][4 V/128] receives the
-// per-tile-quarter argmax keys of every row (see argmax_store).
+// keys != nullptr: fused argmax -- no logits; keys [T][V/16] receives the
+// per-16-row-chunk argmax keys of every row (see argmax_chunk_store).
 ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* logits, void* ws,
                     cudaStream_t s, unsigned long long* keys = nullptr) {
     LmWs w = lm_ws_layout(ws, H, V);
@@ -1271,12 +1282,13 @@ ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* l
         prm.bn = 128;
         prm.offsets = nullptr;
         prm.logits = keys ? nullptr : reinterpret_cast<__nv_bfloat16*>(logits) + static_cast<size_t>(t0) * V;
-        prm.amax_key = keys ? keys + static_cast<size_t>(t0) * 4 * (V / BM) : nullptr;
+        prm.amax_key = keys ? keys + static_cast<size_t>(t0) * (V / 16) : nullptr;
         prm.partials = w.partials;
         prm.status = w.status;
         prm.wait_limit_ns = wait_limit_ns();
         prm.dtrace = g_dtrace;
-        st = launch_stream<LM_STREAM>(K_LM_HEAD, stream_nmax(tc), m, prm, s);
+        // the fused argmax runs the token-major form, which needs all 128 token rows
+        st = launch_stream<LM_STREAM>(K_LM_HEAD, keys ? BM : stream_nmax(tc), m, prm, s);
         if (st != MS_OK) return st;
     }
     return MS_OK;
@@ -1324,7 +1336,7 @@ ms_status verify_keys_launch(const unsigned long long*, int, int, int, const int
 
 extern "C" size_t spec_verify_lm_head_workspace_size(int B, int K, int H, int V) {
     if (B <= 0 || K < 0 || H <= 0 || V <= 0) return 0;
-    return ms::lm_ws_bytes(H, V) + ms::align_up(static_cast<size_t>(B) * (K + 1) * 4 * (V / 128) * 8, 1024);
+    return ms::lm_ws_bytes(H, V) + ms::align_up(static_cast<size_t>(B) * (K + 1) * (V / 16) * 8, 1024);
 }
 
 extern "C" ms_status spec_verify_lm_head_greedy(const void* xhat, const void* w_lm, const int32_t* draft, int B,
@@ -1349,7 +1361,7 @@ extern "C" ms_status spec_verify_lm_head_greedy(const void* xhat, const void* w_
     }
     ms_status st = ms::lm_launch(xhat, w_lm, T, H, V, nullptr, ws, s, keys);
     if (st != MS_OK) return st;
-    return ms::verify_keys_launch(keys, 4 * (V / 128), B, K, draft, argmax, committed, n_committed, s);
+    return ms::verify_keys_launch(keys, V / 16, B, K, draft, argmax, committed, n_committed, s);
 }
 
 extern "C" size_t lm_head_workspace_size(int T, int H, int V) {
