@@ -225,3 +225,45 @@ def moe_layer(a, lw, k: int, bias=None, renormalize: bool = False, eps: float = 
     out = combine(y, ysh, slot, w, a)
     return dict(xhat_bf16=xb, xhat=x, idx=idx, w=w, logits=z, probs=p, offsets=off, perm=perm,
                 slot=slot, y_perm=y, y_shared=ysh, out=out)
+
+
+def fastmtp_draft(h0, tok0, emb, w_proj, w_gate_up, w_down, w_lm, K: int, eps: float = 1e-6):
+    """FastMTP draft block applied recursively for K steps with shared weights
+    (jina.ai, "Modèle et entraînement": one dense draft block reused for every
+    prediction step, trained with recursive hidden-state feedback; the d9249
+    blog's component table: a shared dense draft block, K = 3).
+
+    The pages do not describe the block's inside; this is the multi-token-
+    prediction module of the decoder family it extends, without attention:
+      x   = [bf16(RMSNorm(h)); bf16(RMSNorm(emb[t]))]        (2H)
+      u   = W_proj x                                          (H; W_proj [H, 2H])
+      h'  = u + SwiGLU(bf16(RMSNorm(u)))                      (dense, w_gate_up [2I, H], w_down [H, I])
+      t'  = argmax_v bf16(W_lm bf16(RMSNorm(h')))_v           (the verifier's vocab head; lowest index on ties)
+    starting from the verifier's last hidden state h0 and last committed token
+    tok0, each step feeding (h', t') into the next.
+
+    h0 [B,H] fp32, tok0 [B] int32, emb [V,H] bf16 bits, w_proj [H,2H],
+    w_gate_up [2I,H], w_down [H,I], w_lm [V,H] (bf16 bits or fp32).
+    Returns (drafts [B,K] int32, h_K [B,H] fp32)."""
+    h = _f32(h0)
+    t = _i32(tok0)
+    B, H = h.shape
+    emb = np.ascontiguousarray(emb)
+    wgu = np.ascontiguousarray(w_gate_up)[None]
+    wd = np.ascontiguousarray(w_down)[None]
+    rows = np.arange(B, dtype=np.int32)
+    drafts = np.empty((B, K), np.int32)
+    for i in range(K):
+        _, hb = rmsnorm(h, eps=eps)
+        e = widen_bf16(emb[t]) if emb.dtype == np.uint16 else _f32(emb[t])
+        _, eb = rmsnorm(e, eps=eps)
+        x = np.concatenate([widen_bf16(hb), widen_bf16(eb)], axis=1)
+        u = lm_head(x, w_proj)
+        _, ub = rmsnorm(u, eps=eps)
+        y = expert_ffn_routed(widen_bf16(ub), wgu, wd, np.array([0, B], np.int32), rows, 1)
+        h = combine(y, None, rows[:, None], np.ones((B, 1), np.float32), u)
+        _, xb = rmsnorm(h, eps=eps)
+        z = widen_bf16(bf16_round(lm_head(widen_bf16(xb), w_lm)))
+        t = verify_greedy(z[:, None, :], np.zeros((B, 0), np.int32))[0][:, 0].astype(np.int32)
+        drafts[:, i] = t
+    return drafts, h
