@@ -193,6 +193,30 @@ MS_API ms_status spec_verify_lm_head_greedy(const void* xhat, const void* w_lm, 
                                             int K, int H, int V, int32_t* argmax, int32_t* committed,
                                             int32_t* n_committed, void* ws, size_t ws_bytes, void* stream);
 
+/* FastMTP draft block on the device (jina.ai, "Modèle et entraînement": one
+ * dense draft block applied recursively for K prediction steps, shared
+ * weights, recursive hidden-state feedback).  The pages leave the block's
+ * inside open; this is the multi-token-prediction module without attention:
+ *   x  = [bf16(RMSNorm(h)); bf16(RMSNorm(emb[t]))],  u = W_proj x,
+ *   h' = u + SwiGLU(bf16(RMSNorm(u))),
+ *   t' = argmax bf16(W_lm bf16(RMSNorm(h')))   (lowest index on ties),
+ * starting from the verifier's last hidden state h0 and last committed
+ * token tok0, each step feeding (h', t') into the next; drafts[b,i] = t' of
+ * step i.  RMSNorm: eps 1e-6, no gain.
+ * h0: [B,H] fp32.  tok0: [B] int32.  emb: [V,H] bf16 row-major (not packed).
+ * w_proj: [H,2H], w_gate_up: [2I,H] (gate rows, then up rows), w_down: [H,I],
+ * w_lm: [V,H], all bf16 packed by moe_pack_weights (n = 1).
+ * drafts: [B,K] int32.  h_out: [B,H] fp32, the last hidden state, or NULL;
+ * distinct from h0.  B <= 128, 1 <= K <= 8, H, I, V multiples of 128.  A
+ * token outside [0, V) is flagged MS_ERR_DEVICE_INDEX in the status word at
+ * ws + 0 and its embedding taken as zero.
+ * Scratch: fastmtp_draft_workspace_size(B,H,I,V) bytes. */
+MS_API size_t fastmtp_draft_workspace_size(int B, int H, int I, int V);
+MS_API ms_status fastmtp_draft(const float* h0, const int32_t* tok0, const void* emb, const void* w_proj,
+                               const void* w_gate_up, const void* w_down, const void* w_lm, int B, int H, int I,
+                               int V, int K, int32_t* drafts, float* h_out, void* ws, size_t ws_bytes,
+                               void* stream);
+
 /* Allocation-free variant of spec_verify_greedy.  The pages have no
  * counterpart: this exists for callers that cannot allocate device memory,
  * e.g. a plugin running inside an inference server whose device memory is

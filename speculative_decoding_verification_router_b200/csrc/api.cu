@@ -29,7 +29,7 @@ static const char* kNames[K_COUNT] = {
     "rmsnorm",        "route_rows",      "route_tiled",     "route_cluster", "permute_count", "permute_scatter",
     "ffn_prep",       "gemm1_stream",    "gemm2_stream",    "gemm1_tiled",   "gemm2_tiled",  "ffn_finish",
     "lm_head_stream", "combine",         "verify_partial",  "verify_final",  "verify_cluster", "verify_keys", "wait_probe",
-    "pack_weights"};
+    "pack_weights",   "mtp_prep"};
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kNames[id] : "?"; }
 

@@ -409,6 +409,24 @@ __device__ __forceinline__ uint32_t bf16_order_key(float v) {
 // (t, chunk) of a [T][V/16] table, every slot written exactly once; the
 // verify kernel takes the max over a row's slots: largest value, then lowest
 // index.
+// Fused argmax, vocabulary-major form (small T): the accumulator keeps the
+// vocabulary rows in TMEM lanes, so a token's logits are spread over the 32
+// lanes of each warp.  One warp max over (order key << 16 | 65535 - row) gives
+// the largest value of the warp's 32 rows at its lowest row; it is stored in
+// the first of the two 16-row chunk slots those rows cover, and the second
+// slot gets 0, which every real key exceeds.  Called by all 32 lanes.
+__device__ __forceinline__ void argmax_warp_store(unsigned long long* keys, int ld, int t, float v, int row_in_tile,
+                                                  int tile, int quad, int lane) {
+    uint32_t k32 = (bf16_order_key(v) << 16) | (0xFFFFu - static_cast<uint32_t>(row_in_tile));
+    k32 = __reduce_max_sync(0xffffffffu, k32);
+    if (lane == 0) {
+        const uint32_t idx = static_cast<uint32_t>(tile) * BM + (0xFFFFu - (k32 & 0xFFFFu));
+        unsigned long long* slot = keys + static_cast<size_t>(t) * ld + tile * (BM / 16) + quad * 2;
+        slot[0] = (static_cast<unsigned long long>(k32 >> 16) << 32) | (0xFFFFFFFFu - idx);
+        slot[1] = 0;
+    }
+}
+
 __device__ __forceinline__ void argmax_chunk_store(unsigned long long* keys, int ld, int t, const float (&v)[16],
                                                    int chunk) {
     uint32_t best = 0;
@@ -526,7 +544,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     constexpr bool kStream = Cfg<MODE>::kStream;
     constexpr int kSub = Cfg<MODE>::kSub;
     // vocab head with the fused argmax: tokens are the MMA's M operand, vocabulary rows its N
-    const bool tokM = MODE == LM_STREAM && p.amax_key != nullptr;
+    // (only with a 128-token operand; with fewer tokens the fused argmax keeps the vocabulary rows in M)
+    const bool tokM = MODE == LM_STREAM && p.amax_key != nullptr && NMAX == BM;
+    const bool vocM = MODE == LM_STREAM && p.amax_key != nullptr && NMAX < BM;
     constexpr bool kG1 = Cfg<MODE>::kG1;
     constexpr int ST = L::STAGES;
 
@@ -847,6 +867,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         if (r_in < rows) argmax_chunk_store(p.amax_key, p.V / 16, r_in, va, w.n * (BM / 16) + ch);
                         continue;
                     }
+                    if (vocM) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (ch * 16 + j < rows)
+                                argmax_warp_store(p.amax_key, p.V / 16, ch * 16 + j, va[j], r_in, w.n, q4, lane);
+                        continue;
+                    }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int t = ch * 16 + j;
@@ -967,7 +994,8 @@ __global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p)
     if (c_first == c_last) return;   // one CTA did the whole tile and stored it
     const int rows = sched.rows[g], row0 = sched.row0[g];
     const int ch = blockIdx.y;
-    if (!(MODE == LM_STREAM && p.amax_key) && ch * 16 >= rows) return;   // (argmax mode: ch = vocabulary rows)
+    // (token-major argmax: ch = 16 vocabulary rows, all of them)
+    if (!(MODE == LM_STREAM && p.amax_key && NMAX == BM) && ch * 16 >= rows) return;
     constexpr bool kG1 = Cfg<MODE>::kG1;
     const int slot_floats = BM * NMAX * (kG1 ? 2 : 1);
     const int r = threadIdx.x;
@@ -979,6 +1007,18 @@ __global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p)
     float va[16], vb[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) va[j] = vb[j] = 0.f;
+    if (MODE == LM_STREAM && p.amax_key && NMAX < BM) {
+        // vocabulary-major partials: thread = row r, chunk ch = 16 tokens
+        const int rc = rows - ch * 16;
+        if (rc <= 4) slot_sum_col<1>(slot_of, c_first, c_last, ch, r, va);
+        else if (rc <= 8) slot_sum_col<2>(slot_of, c_first, c_last, ch, r, va);
+        else slot_sum_col<4>(slot_of, c_first, c_last, ch, r, va);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (ch * 16 + j < rows) argmax_warp_store(p.amax_key, p.V / 16, ch * 16 + j, va[j], r, n, r >> 5, r & 31);
+        fin_stamp<MODE>(p, TS_EXIT);
+        return;
+    }
     if (MODE == LM_STREAM && p.amax_key) {
         // token-major partials: thread = token, chunk ch = 16 vocabulary rows
         if (r < rows) {
@@ -1264,8 +1304,9 @@ size_t lm_ws_bytes(int H, int V) { return lm_ws_layout(nullptr, H, V).bytes; }
 // keys != nullptr: fused argmax -- no logits; keys [T][V/16] receives the
 // per-16-row-chunk argmax keys of every row (see argmax_chunk_store).
 ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* logits, void* ws,
-                    cudaStream_t s, unsigned long long* keys = nullptr) {
+                    cudaStream_t s, unsigned long long* keys = nullptr, int32_t* status = nullptr) {
     LmWs w = lm_ws_layout(ws, H, V);
+    if (status) w.status = status;
     for (int t0 = 0; t0 < T; t0 += BM) {
         const int tc = T - t0 < BM ? T - t0 : BM;
         const __nv_bfloat16* xc = reinterpret_cast<const __nv_bfloat16*>(x) + static_cast<size_t>(t0) * H;
@@ -1287,11 +1328,42 @@ ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* l
         prm.status = w.status;
         prm.wait_limit_ns = wait_limit_ns();
         prm.dtrace = g_dtrace;
-        // the fused argmax runs the token-major form, which needs all 128 token rows
-        st = launch_stream<LM_STREAM>(K_LM_HEAD, keys ? BM : stream_nmax(tc), m, prm, s);
+        // the fused argmax: token-major form (all 128 token rows) above 32 tokens,
+        // vocabulary-major with warp maxima below
+        st = launch_stream<LM_STREAM>(K_LM_HEAD, keys && tc > 32 ? BM : stream_nmax(tc), m, prm, s);
         if (st != MS_OK) return st;
     }
     return MS_OK;
+}
+
+// ------------------------------------------------------------ linear layer
+// y [T][N] fp32 = x [T][K] . W^T for T <= 128, run as the streaming GEMM2
+// schedule with one group (weights are the M operand, the T token rows the N
+// operand; split tiles finished by ffn_finish_kernel).  x: bf16 with x_rows
+// >= T rows allocated, W: packed [N][K], offsets: device {0, T}.  Scratch:
+// linear_ws_bytes(T) for the split-tile partials; status: device word.
+size_t linear_ws_bytes(int T) {
+    return align_up(static_cast<size_t>(BM) * stream_nmax(T) * 2 * sizeof(float) * 4 * num_sms(), 1024);
+}
+
+ms_status linear_launch(const void* x, int x_rows, int T, int K, const void* w, int N, const int32_t* offsets,
+                        float* y, void* ws, int32_t* status, cudaStream_t s) {
+    if (T > BM || K % 128 != 0 || N % 128 != 0) return MS_ERR_UNSUPPORTED;
+    Params prm{};
+    prm.T = T; prm.H = N; prm.E = 1; prm.I = K; prm.S = 0; prm.k = 1; prm.V = 0;
+    prm.bn = 128;
+    prm.offsets = offsets;
+    prm.y_perm = y;
+    prm.y_bf16 = 0;
+    prm.partials = static_cast<float*>(ws);
+    prm.status = status;
+    prm.wait_limit_ns = wait_limit_ns();
+    prm.dtrace = g_dtrace;
+    Maps m{};
+    if (!make_packed_map(&m.w_a, w, N, K, 1) || !make_map(&m.tok_r, x, K, x_rows, 1, TOKBOX)) return MS_ERR_CUDA;
+    m.w_s = m.w_a;
+    m.tok_s = m.tok_r;
+    return launch_stream<G2_STREAM>(K_GEMM2_STREAM, stream_nmax(T), m, prm, s);
 }
 
 }  // namespace ms

@@ -34,6 +34,7 @@ enum KernelId : int {
     K_VERIFY_KEYS,
     K_WAIT_PROBE,
     K_PACK,
+    K_MTP_PREP,
     K_COUNT
 };
 const char* kernel_name(int id);

@@ -49,6 +49,8 @@ def _load():
         "spec_verify_workspace_size": (Z, [I, I, I]),
         "spec_verify_greedy": (I, [P, I, P, I, I, I, P, P, P, P, Z, P]),
         "spec_verify_lm_head_workspace_size": (Z, [I, I, I, I]),
+        "fastmtp_draft_workspace_size": (Z, [I, I, I, I]),
+        "fastmtp_draft": (I, [P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, Z, P]),
         "spec_verify_lm_head_greedy": (I, [P, P, P, I, I, I, I, P, P, P, P, Z, P]),
         "moe_layer_workspace_size": (Z, [I, I, I, I, I, I]),
         "moe_layer_forward": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, Z, P]),
@@ -269,6 +271,27 @@ def verify_lm_head_greedy(xhat, w_lm, draft, ws: Optional[Workspace] = None, out
     _check(_lib.spec_verify_lm_head_greedy(_p(xhat), _p(w_lm), _p(draft), B, K, H, V, _p(am), _p(cm), _p(n),
                                            w.c(), w.nbytes, _stream(stream)), "spec_verify_lm_head_greedy")
     return am, cm, n
+
+
+def fastmtp_draft(h0, tok0, emb, w_proj, w_gate_up, w_down, w_lm, K: int, ws: Optional[Workspace] = None,
+                  out=None, stream=None):
+    """FastMTP draft block applied K times on the device.  h0 [B,H] fp32, tok0 [B]
+    int32, emb [V,H] bf16 (row-major), w_proj [H,2H], w_gate_up [2I,H], w_down [H,I],
+    w_lm [V,H] bf16 packed by pack_weights.  Returns (drafts [B,K] int32, h_out [B,H] fp32)."""
+    _dev(h0, torch.float32, "h0")
+    _dev(tok0, torch.int32, "tok0")
+    for name, t in (("emb", emb), ("w_proj", w_proj), ("w_gate_up", w_gate_up), ("w_down", w_down), ("w_lm", w_lm)):
+        _dev(t, torch.bfloat16, name)
+    B, H = h0.shape
+    V = emb.shape[0]
+    I = w_down.shape[-1]
+    dev = h0.device
+    drafts, h_out = out if out is not None else (torch.empty((B, K), dtype=torch.int32, device=dev),
+                                                 torch.empty((B, H), dtype=torch.float32, device=dev))
+    w = _ws(ws, _lib.fastmtp_draft_workspace_size(B, H, I, V), dev)
+    _check(_lib.fastmtp_draft(_p(h0), _p(tok0), _p(emb), _p(w_proj), _p(w_gate_up), _p(w_down), _p(w_lm), B, H, I,
+                              V, K, _p(drafts), _p(h_out), w.c(), w.nbytes, _stream(stream)), "fastmtp_draft")
+    return drafts, h_out
 
 
 def layer_workspace_size(T, H, E, I, S, k) -> int:
