@@ -549,13 +549,53 @@ def run_k_sweep(args, rank, world, local):
     replayed.  Reports per K the step time, tau (tokens committed per sequence
     per step, from the verification of drafts that match w.p. p_match), the
     spec-step cost c(K) = t_step(K) / t_step(0) in plain-decoding steps, and
-    the speedup tau / c over plain greedy decoding."""
+    the speedup tau / c over plain greedy decoding -- and the same with the
+    time of the on-device FastMTP draft block for K steps added to the step."""
     import dataclasses
     import torch
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     dist = init_dist(world, "nccl")
     base = synth.STEP_B32
+    from speculative_decoding_verification_router_b200 import moespec as ms
+    # the FastMTP draft block (dense width = the MoE layer's active width) with
+    # the verifier's vocabulary size; its own seeded random weights
+    g = torch.Generator(device=device)
+    g.manual_seed(4321 + rank)
+    rnd = lambda shape, std: (torch.randn(shape, generator=g, device=device) * std).to(torch.bfloat16)
+    Bd, Hd, Id, Vd = base.B, base.H, (base.k + base.S) * base.I, base.V
+    draft_w = dict(emb=rnd((Vd, Hd), 1.0), w_proj=ms.pack_weights(rnd((Hd, 2 * Hd), base.weight_std)),
+                   w_gate_up=ms.pack_weights(rnd((1, 2 * Id, Hd), base.weight_std)),
+                   w_down=ms.pack_weights(rnd((1, Hd, Id), base.weight_std)),
+                   w_lm=ms.pack_weights(rnd((Vd, Hd), base.weight_std)))
+    h0 = torch.randn((Bd, Hd), generator=g, device=device)
+    tok0 = torch.randint(0, Vd, (Bd,), generator=g, device=device, dtype=torch.int32)
+    dws = ms.Workspace(ms.lib().fastmtp_draft_workspace_size(Bd, Hd, Id, Vd), device)
+
+    def time_draft(K):
+        out = (torch.empty((Bd, K), dtype=torch.int32, device=device),
+               torch.empty((Bd, Hd), dtype=torch.float32, device=device))
+        st = torch.cuda.Stream(device)
+        call = lambda: ms.fastmtp_draft(h0, tok0, draft_w["emb"], draft_w["w_proj"], draft_w["w_gate_up"],
+                                        draft_w["w_down"], draft_w["w_lm"], K, ws=dws, out=out)
+        with torch.cuda.stream(st):
+            for _ in range(3):
+                call()
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=st):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(10, args.steps // 4)
+        with torch.cuda.stream(st):
+            e0.record(st)
+            for _ in range(reps):
+                gr.replay()
+            e1.record(st)
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), world, device) / reps
+
     sampler = ClockSampler(local)
     sampler.start()
     rows = []
@@ -588,7 +628,8 @@ def run_k_sweep(args, rank, world, local):
         t_ms = max_over_ranks(ev0.elapsed_time(ev1), world, device) / args.steps
         n = prob.vout[2].cpu().numpy()
         tau = float(n.mean())
-        rows.append({"K": K, "ms_per_step": round(t_ms, 5), "tau": round(tau, 4),
+        t_draft = time_draft(K) if K > 0 else 0.0
+        rows.append({"K": K, "ms_per_step": round(t_ms, 5), "draft_ms": round(t_draft, 5), "tau": round(tau, 4),
                      "tau_closed_form": round(metrics.expected_tau_iid(shp.p_match, K), 4) if K else 1.0,
                      "committed_tok_s": round(shp.B * tau / (t_ms / 1e3) * world, 1)})
         del graph, prob
@@ -598,6 +639,9 @@ def run_k_sweep(args, rank, world, local):
     for r in rows:
         r["c"] = round(r["ms_per_step"] / t0, 4)
         r["speedup"] = round(r["tau"] / r["c"], 4)
+        # with the on-device FastMTP draft of the same K in the loop
+        r["c_with_draft"] = round((r["ms_per_step"] + r["draft_ms"]) / t0, 4)
+        r["speedup_with_draft"] = round(r["tau"] / r["c_with_draft"], 4)
     best = max(rows, key=lambda r: r["speedup"])
     return {"metric": "speedup of the 12-layer speculative decode step over plain greedy decoding, K swept 0..3",
             "value": rows[-1]["speedup"], "unit": "x (K=3)", "n_gpus": world, "steps": args.steps,
@@ -606,7 +650,9 @@ def run_k_sweep(args, rank, world, local):
             "config": {"workload": base.name, "B": base.B, "layers": base.layers, "V": base.V,
                        "p_match": base.p_match, "graph": "one CUDA graph per K, replayed",
                        "vocab_head": "fused" if args.fused_head else "unfused",
-                       "l2": "12 distinct weight sets (5.5 GB) > 126 MB L2"},
+                       "l2": "12 distinct weight sets (5.5 GB) > 126 MB L2",
+                       "draft_block": {"H": Hd, "I": Id, "V": Vd, "note": "random weights: timed, tau from the "
+                                       "synthetic drafts, not from the draft block"}},
             "best_K": best["K"], "sweep": rows, "clocks": sampler.summary()}
 
 
