@@ -22,6 +22,7 @@ Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import os
@@ -271,6 +272,10 @@ def run_ours(args, rank, world, local):
     from speculative_decoding_verification_router_b200 import moespec as ms
 
     shp = WORKLOADS[args.workload]
+    if args.tokens:
+        if shp.tokens is None:
+            raise SystemExit("--tokens applies to the prefill workload")
+        shp = dataclasses.replace(shp, name=f"prefill_t{args.tokens}_h{shp.H}_e{shp.E}", tokens=args.tokens)
     n_sets = args.sets or {"verify_b1": 4, "verify_b32": 4, "step12_b32": 12, "prefill": 1}[args.workload]
     prob = Problem(shp, n_sets, seed=1234 + rank, device=device, fused_head=args.fused_head)
     stream = torch.cuda.Stream(device)
@@ -666,6 +671,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sets", type=int, default=0, help="distinct weight sets rotated across steps (0 = workload default)")
+    ap.add_argument("--tokens", type=int, default=0, help="prefill workload: token count (a smaller case to profile)")
     ap.add_argument("--k-sweep", action="store_true",
                     help="12-layer step at B=32 for K = 0..3: step time, tau, spec-step cost and speedup")
     ap.add_argument("--fused-head", action="store_true",

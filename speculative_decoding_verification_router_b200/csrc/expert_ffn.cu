@@ -64,6 +64,7 @@ struct Maps {
 struct Params {
     int T, H, E, I, S, k, V;
     int bn;                        // tiled GEMM2 output tile width (256 or 128)
+    int mt;                        // tiled: token rows per work tile (128, or 256 for a CTA pair; 0 = 128)
     const int32_t* offsets;        // [E+1]; nullptr for the vocab head
     __nv_bfloat16* h_perm;         // [rows][I]
     __nv_bfloat16* h_sh;           // [T][S*I]
@@ -196,7 +197,8 @@ __device__ void build_schedule_n(const Params& p, Sched& s) {
                 tiles = group_ntiles<MODE>(p, g);
                 units = tiles * group_ktiles<MODE>(p, g);
             } else {
-                units = ((rows + BM - 1) / BM) * group_ntiles<MODE>(p, g);
+                const int mt = p.mt ? p.mt : BM;
+                units = ((rows + mt - 1) / mt) * group_ntiles<MODE>(p, g);
             }
         }
         s.prefix[g + 1] = units;   // scanned below
@@ -366,7 +368,7 @@ struct WorkIter {
             const int m = local / nt;
             w.g = g;
             w.n = local - m * nt;
-            w.m0 = m * BM;
+            w.m0 = m * (p.mt ? p.mt : BM);
             w.k0 = 0;
             w.kt = group_ktiles<MODE>(p, g);
             w.k1 = w.kt;
@@ -954,6 +956,279 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (threadIdx.x == 32) tstamp(p, MODE, TS_EXIT);
 }
 
+// ------------------------------------------------------------ tiled GEMMs on CTA pairs
+// The prefill contractions as 256 x 256 tiles on a pair of CTAs (a cluster of
+// two, tcgen05 cta_group::2).  Each CTA stages 128 token rows and its half of
+// the tile's 256 weight rows (GEMM1: CTA 0 the gate rows, CTA 1 the up rows of
+// the same 128 features; GEMM2: 128 of the 256 output features), so a CTA
+// pulls 32 KB per 64-wide k-step instead of 48 KB and keeps six stages in
+// flight; the first CTA issues one M = 256, N = 256 MMA per 16-wide k-slice
+// and each CTA's TMEM receives its 128 token rows x 256 columns.
+//   - both CTAs' loads complete on CTA 0's `full` barrier (armed by CTA 0
+//     for the pair's bytes), on which CTA 0's MMA thread waits; its commits
+//     arrive on `empty` (stage free) and `tfull` (accumulator ready) in both
+//     CTAs;
+//   - both CTAs' epilogue warps arrive on CTA 0's `tempty` (count 8).
+// No TMA multicast: every load reads this GPU's memory into its own CTA.
+constexpr int PAIR_STAGE = 2 * TILE_BYTES;   // 128 token rows + 128 weight rows, 64 wide
+constexpr int PAIR_ST = 6;
+constexpr int PAIR_SMEM = PAIR_ST * PAIR_STAGE + 1024;
+
+template <int MODE>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    ffn_gemm_pair_kernel(const __grid_constant__ Maps maps, const Params p) {
+    static_assert(MODE == G1_TILED || MODE == G2_TILED, "CTA pairs run the tiled schedule");
+    constexpr int ST = PAIR_ST;
+    extern __shared__ uint8_t dsmem[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t bar_full[ST], bar_empty[ST], bar_tfull[2], bar_tempty[2], bar_drain;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ volatile int abort_sh;
+    __shared__ int go_sh[2];
+    __shared__ Sched sched;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t rank = cluster_rank();          // 0: issues the MMAs
+    const int pc = static_cast<int>(blockIdx.x >> 1), npair = static_cast<int>(gridDim.x >> 1);
+    const uint64_t lim = p.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        tstamp(p, MODE, TS_ENTRY);
+        tma_prefetch_map(&maps.w_a);
+        tma_prefetch_map(&maps.w_s);
+        tma_prefetch_map(&maps.tok_r);
+        tma_prefetch_map(&maps.tok_s);
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(smem_addr(&bar_full[i]), 1);
+            mbar_init(smem_addr(&bar_empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_addr(&bar_tfull[i]), 1);
+            mbar_init(smem_addr(&bar_tempty[i]), 8);
+        }
+        mbar_init(smem_addr(&bar_drain), 1);
+        abort_sh = 0;
+        fence_mbar_init();
+    }
+    build_schedule<MODE>(p, sched);
+    grid_dep_wait();
+    // both CTAs' barriers exist before either CTA signals the other's
+    cluster_sync_all();
+    if (warp == 1) {
+        tmem_alloc_pair(smem_addr(&tmem_base_sh), TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    grid_dep_launch();
+    const uint32_t tmem_base = tmem_base_sh;
+    if (threadIdx.x == 0) tstamp(p, MODE, TS_SETUP);
+    const int kt_h = p.H / BK, kt_i = p.I / BK;
+
+    if (warp == 0) {
+      if (lane == 0) {
+        // ---------------------------------------------------- TMA producer (this CTA's halves)
+        bool ok = true;
+        int q = 0;
+        const uint32_t full0 = mapa_shared(smem_addr(&bar_full[0]), 0);
+        WorkIter<MODE> it;
+        it.init(p, sched, pc, npair);
+        Work w;
+        while (ok && it.next(p, sched, w)) {
+            const bool shared = p.offsets != nullptr && w.g == p.E;
+            const CUtensorMap* tm = shared ? &maps.tok_s : &maps.tok_r;
+            const int trow = sched.row0[w.g] + w.m0 + static_cast<int>(rank) * BM;
+            for (int kt = w.k0; kt < w.k1; ++kt, ++q) {
+                const int stage = q % ST;
+                const uint32_t phase = static_cast<uint32_t>(q / ST) & 1u;
+                if (!mbar_wait(smem_addr(&bar_empty[stage]), phase ^ 1u, lim, &abort_sh)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t a = sbase + stage * PAIR_STAGE, b = a + TILE_BYTES;
+                // both CTAs' loads complete on CTA 0's `full` barrier, which
+                // CTA 0's producer arms for the pair's 64 KB
+                const uint32_t full = full0 + stage * 8;
+                if (rank == 0) mbar_expect_tx(smem_addr(&bar_full[stage]), 2 * PAIR_STAGE);
+                tma_load_3d_pair(a, tm, full, kt * BK, trow, 0);
+                if (MODE == G1_TILED) {
+                    int z = w.g, fl = w.n * BM;
+                    const CUtensorMap* wm = &maps.w_a;
+                    if (shared) { z = fl / p.I; fl -= z * p.I; wm = &maps.w_s; }
+                    tma_load_3d_pair(b, wm, full, 0, packed_row(rank == 0 ? fl : p.I + fl, kt, kt_h), z);
+                } else {
+                    const int n0 = w.n * 2 * BM + static_cast<int>(rank) * BM;
+                    if (shared) {
+                        const int kx = kt * BK, z = kx / p.I;
+                        tma_load_3d_pair(b, &maps.w_s, full, 0, packed_row(n0, (kx - z * p.I) / BK, kt_i), z);
+                    } else {
+                        tma_load_3d_pair(b, &maps.w_a, full, 0, packed_row(n0, kt, kt_i), w.g);
+                    }
+                }
+            }
+        }
+        if (!ok) {
+            report_status(p.status, MS_ERR_TIMEOUT);
+            abort_sh = 1;
+        }
+        // drain: every load this thread issued has landed once CTA 0's MMAs
+        // released its stage (they waited for the full pair of loads)
+        for (int s2 = 0; s2 < ST && s2 < q; ++s2) {
+            const int q_last = s2 + ((q - 1 - s2) / ST) * ST;
+            volatile int never = 0;
+            if (!mbar_wait(smem_addr(&bar_empty[s2]), static_cast<uint32_t>(q_last / ST) & 1u, lim, &never))
+                report_status(p.status, MS_ERR_TIMEOUT);
+        }
+        tstamp(p, MODE, TS_PRODUCER_DONE);
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      if (lane == 0) {
+        if (rank == 0) {
+            bool ok = true;
+            WorkIter<MODE> it;
+            it.init(p, sched, pc, npair);
+            Work w;
+            // ---------------------------------------------------- MMA issuer (one thread of CTA 0)
+            const uint32_t idesc = idesc_bf16_f32(2 * BM, 2 * BM);
+            int q = 0, acc = 0;
+            uint32_t acc_phase = 0;
+            while (ok && it.next(p, sched, w)) {
+                if (!mbar_wait(smem_addr(&bar_tempty[acc]), acc_phase ^ 1u, lim, &abort_sh)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + acc * 256;
+                for (int kt = w.k0; kt < w.k1; ++kt, ++q) {
+                    const int stage = q % ST;
+                    const uint32_t phase = static_cast<uint32_t>(q / ST) & 1u;
+                    if (!mbar_wait(smem_addr(&bar_full[stage]), phase, lim, &abort_sh)) {
+                        ok = false;
+                        break;
+                    }
+                    if (q == 0) tstamp(p, MODE, TS_FIRST_DATA);
+                    tc_fence_after();
+                    const uint32_t a = sbase + stage * PAIR_STAGE, b = a + TILE_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_bf16_pair(d0, smem_desc_sw128(a + kk * 32), smem_desc_sw128(b + kk * 32), idesc,
+                                      (kt > w.k0 || kk > 0) ? 1u : 0u);
+                    mma_commit_pair(smem_addr(&bar_empty[stage]), 0x3);
+                }
+                if (!ok) break;
+                mma_commit_pair(smem_addr(&bar_tfull[acc]), 0x3);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok) {
+                report_status(p.status, MS_ERR_TIMEOUT);
+                abort_sh = 1;
+            }
+            tstamp(p, MODE, TS_LAST_MMA);
+            // drain: every pair MMA issued by this thread completes before TMEM is freed
+            mma_commit_pair(smem_addr(&bar_drain), 0x1);
+            volatile int never = 0;
+            if (!mbar_wait(smem_addr(&bar_drain), 0, lim, &never)) report_status(p.status, MS_ERR_TIMEOUT);
+        }
+      }
+      __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue (4 warps, this CTA's 128 rows)
+        const int q4 = warp & 3;
+        const int r_in = q4 * 32 + lane;
+        const int etid = threadIdx.x - 64;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        const int ldh_r = p.I, ldh_s = p.S * p.I;
+        const uint32_t tempty0 = mapa_shared(smem_addr(&bar_tempty[0]), 0);
+        auto tmem_at = [&](int col) -> uint32_t {
+            return tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) + static_cast<uint32_t>(acc * 256 + col);
+        };
+        WorkIter<MODE> it;
+        it.init(p, sched, pc, npair);
+        Work w;
+        while (ok && it.next(p, sched, w)) {
+            if (!epi_wait(smem_addr(&bar_tfull[acc]), acc_phase, lim, &abort_sh, etid, go_sh[acc])) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int g = w.g;
+            const bool shared = p.offsets != nullptr && g == p.E;
+            const int rows = sched.rows[g], row0 = sched.row0[g];
+            const int rr = w.m0 + static_cast<int>(rank) * BM + r_in;   // row within the group
+            const bool valid = rr < rows;
+            const size_t orow = static_cast<size_t>(shared ? rr : row0 + rr);
+            if (MODE == G1_TILED) {
+                const int f0 = w.n * BM;
+                __nv_bfloat16* dst = shared ? p.h_sh + orow * ldh_s + f0 : p.h_perm + orow * ldh_r + f0;
+                for (int ch = 0; ch < BM / 16; ++ch) {
+                    float g16[16], u16[16];
+                    tmem_ld16(tmem_at(ch * 16), g16);
+                    tmem_ld16(tmem_at(128 + ch * 16), u16);
+                    tmem_ld_wait();
+                    if (valid) {
+                        __align__(16) __nv_bfloat162 hb[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            hb[j] = __floats2bfloat162_rn(silu_mul(g16[2 * j], u16[2 * j]),
+                                                          silu_mul(g16[2 * j + 1], u16[2 * j + 1]));
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 16);
+                        d4[0] = reinterpret_cast<const uint4*>(hb)[0];
+                        d4[1] = reinterpret_cast<const uint4*>(hb)[1];
+                    }
+                }
+            } else {
+                const int n0 = w.n * 2 * BM;
+                for (int ch = 0; ch < 2 * BM / 16; ++ch) {
+                    float v16[16];
+                    tmem_ld16(tmem_at(ch * 16), v16);
+                    tmem_ld_wait();
+                    if (!valid) continue;
+                    if (shared || !p.y_bf16) {
+                        float* dst = shared ? p.y_sh + orow * p.H + n0 + ch * 16
+                                            : reinterpret_cast<float*>(p.y_perm) + orow * p.H + n0 + ch * 16;
+                        float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            d4[j] = make_float4(v16[4 * j], v16[4 * j + 1], v16[4 * j + 2], v16[4 * j + 3]);
+                    } else {
+                        __align__(16) __nv_bfloat162 hb[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) hb[j] = __floats2bfloat162_rn(v16[2 * j], v16[2 * j + 1]);
+                        uint4* d4 = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.y_perm) +
+                                                             orow * p.H + n0 + ch * 16);
+                        d4[0] = reinterpret_cast<const uint4*>(hb)[0];
+                        d4[1] = reinterpret_cast<const uint4*>(hb)[1];
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(smem_addr(&bar_tempty[acc]));
+                else mbar_arrive_remote(tempty0 + acc * 8);
+            }
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+        if (!ok) {
+            if (etid == 0) report_status(p.status, MS_ERR_TIMEOUT);
+            abort_sh = 1;
+        }
+        if (etid == 0) tstamp(p, MODE, TS_EPI_DONE);
+    }
+    tc_fence_before();
+    __syncthreads();
+    // CTA 0's last MMAs read this CTA's shared memory and write its TMEM: neither
+    // CTA frees either before both got here
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    if (threadIdx.x == 32) tstamp(p, MODE, TS_EXIT);
+}
+
 // ------------------------------------------------------------ finish kernel
 // Sums the parts of every tile the streaming GEMM split between CTAs (its
 // contributors wrote fp32 partials and moved on) in CTA order, and applies
@@ -1076,29 +1351,30 @@ __global__ void __launch_bounds__(256) ffn_prep_kernel(const __nv_bfloat16* __re
                                                        int t_pad, int32_t* status) {
     grid_dep_wait();
     grid_dep_launch();
+    // one warp per output row: the row's token id is read once, then the warp
+    // copies the row in 16-byte pieces (a 2,560-byte row is 5 per lane)
+    const int lane = threadIdx.x & 31;
     const int n8 = H / 8;
-    const long stride = static_cast<long>(gridDim.x) * blockDim.x;
-    const long tid = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x;
-    const long n_perm = static_cast<long>(rows_pad) * n8;
-    for (long v = tid; v < n_perm; v += stride) {
-        const int r = static_cast<int>(v / n8), c = static_cast<int>(v % n8);
-        uint4 val = make_uint4(0, 0, 0, 0);
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const int warp0 = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    for (int r = warp0; r < rows_pad; r += nwarps) {
+        int t = -1;
         if (r < rows) {
-            const int t = __ldg(perm + r);
-            if (t >= 0 && t < T)
-                val = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H) + c);
-            else
-                report_status(status, MS_ERR_DEVICE_INDEX);
+            t = __ldg(perm + r);
+            if (t < 0 || t >= T) {
+                if (lane == 0) report_status(status, MS_ERR_DEVICE_INDEX);
+                t = -1;
+            }
         }
-        reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(r) * H)[c] = val;
+        const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t < 0 ? 0 : t) * H);
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(r) * H);
+        for (int c = lane; c < n8; c += 32) dst[c] = t >= 0 ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
     }
     if (x_pad) {
-        const long n_pad = static_cast<long>(t_pad) * n8;
-        for (long v = tid; v < n_pad; v += stride) {
-            const int r = static_cast<int>(v / n8), c = static_cast<int>(v % n8);
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (r < T) val = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * H) + c);
-            reinterpret_cast<uint4*>(x_pad + static_cast<size_t>(r) * H)[c] = val;
+        for (int r = warp0; r < t_pad; r += nwarps) {
+            const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(r < T ? r : 0) * H);
+            uint4* dst = reinterpret_cast<uint4*>(x_pad + static_cast<size_t>(r) * H);
+            for (int c = lane; c < n8; c += 32) dst[c] = r < T ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
         }
     }
 }
@@ -1156,6 +1432,49 @@ static ms_status launch_gemm(int id, const Maps& maps, const Params& prm, cudaSt
     return launch(id, ffn_gemm_kernel<MODE, NMAX>, dim3(num_sms()), dim3(NTHREADS), L::SMEM, s, maps, prm);
 }
 
+// The tiled GEMM on CTA pairs: as many pairs as can be resident at once (at
+// most one CTA per SM), 0 if the device cannot place any.
+template <int MODE>
+static int pair_grid() {
+    static int grid = -1;
+    if (grid < 0) {
+        grid = 0;
+        if (cudaFuncSetAttribute(ffn_gemm_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 PAIR_SMEM) != cudaSuccess ||
+            cudaFuncSetAttribute(ffn_gemm_pair_kernel<MODE>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            return grid;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(num_sms());
+        cfg.blockDim = dim3(NTHREADS);
+        cfg.dynamicSmemBytes = PAIR_SMEM;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, ffn_gemm_pair_kernel<MODE>, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            nclusters = 0;
+        }
+        const int cap = num_sms() / 2;
+        grid = 2 * (nclusters < cap ? nclusters : cap);
+    }
+    return grid;
+}
+
+template <int MODE>
+static ms_status launch_gemm_pair(int id, const Maps& maps, Params prm, cudaStream_t s) {
+    prm.mt = 2 * BM;
+    return launch_cluster(id, ffn_gemm_pair_kernel<MODE>, dim3(pair_grid<MODE>()), dim3(NTHREADS), PAIR_SMEM, s, 2,
+                          maps, prm);
+}
+
 template <int MODE, int NMAX>
 static ms_status launch_stream_n(int id, const Maps& maps, Params prm, cudaStream_t s) {
     prm.nct = num_sms();
@@ -1175,6 +1494,16 @@ static ms_status launch_stream(int id, int nmax, const Maps& maps, const Params&
         case 64: return launch_stream_n<MODE, 64>(id, maps, prm, s);
         default: return launch_stream_n<MODE, 128>(id, maps, prm, s);
     }
+}
+
+// MOESPEC_NO_PAIR=1 runs the prefill GEMMs on single CTAs (for comparison).
+static bool pair_off() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("MOESPEC_NO_PAIR");
+        v = (e && e[0] == '1') ? 1 : 0;
+    }
+    return v == 1;
 }
 
 static uint64_t* g_dtrace = nullptr;
@@ -1228,10 +1557,10 @@ ms_status ffn_launch(const void* x, const int32_t* offsets, const int32_t* perm,
     FfnWs w = ffn_ws_layout(ws, T, H, E, I, S, k);
     const bool stream = T <= 128;
     const int rows = T * k;
-    // 1. gather + pad
+    // 1. gather + pad (one warp per row, 8 rows per block)
     {
-        const long work = static_cast<long>(w.rows_pad) * (H / 8);
-        const int grid = static_cast<int>(work / 256 + 1 < 4L * num_sms() ? work / 256 + 1 : 4L * num_sms());
+        const long want = (static_cast<long>(w.rows_pad) + 7) / 8;
+        const int grid = static_cast<int>(want < 8L * num_sms() ? want : 8L * num_sms());
         ms_status st = launch(K_FFN_PREP, ffn_prep_kernel, dim3(grid), dim3(256), 0, s,
                               reinterpret_cast<const __nv_bfloat16*>(x), perm, T, H, rows, w.rows_pad,
                               w.x_perm, stream ? w.x_pad : static_cast<__nv_bfloat16*>(nullptr), w.t_pad,
@@ -1270,8 +1599,13 @@ ms_status ffn_launch(const void* x, const int32_t* offsets, const int32_t* perm,
         if (st1 != MS_OK) return st1;
         return launch_stream<G2_STREAM>(K_GEMM2_STREAM, stream_nmax(T), m2, prm, s);
     }
+    // prefill.  GEMM2 runs as 256 x 256 tiles on CTA pairs when the output width
+    // splits in 256s (measured 638 vs 789 us at 36,992 tokens); GEMM1 stays on
+    // single CTAs, where the pair form measured slower (1,264 vs 1,212 us).
     ms_status st = launch_gemm<G1_TILED, 16>(K_GEMM1_TILED, m1, prm, s);
     if (st != MS_OK) return st;
+    if (prm.bn == 256 && !pair_off() && pair_grid<G2_TILED>() >= 2)
+        return launch_gemm_pair<G2_TILED>(K_GEMM2_TILED, m2, prm, s);
     return launch_gemm<G2_TILED, 16>(K_GEMM2_TILED, m2, prm, s);
 }
 

@@ -99,10 +99,23 @@ __global__ void __launch_bounds__(256) route_rows_kernel(const __nv_bfloat16* __
                           w + static_cast<size_t>(t) * k, lane);
 }
 
-// Large T (E <= 64): 64 tokens x 64 experts per block, register tile 4x4 per
-// thread, H walked in chunks of 32 through shared memory; then top-k per
-// token from the logits kept in shared memory.
-constexpr int RT_TOK = 64, RT_EXP = 64, RT_K = 32, RT_PAD = 4;
+// Large T (E <= 64): 128 tokens x 64 experts per block of 256 threads, an
+// 8 x 4 register tile per thread, H walked in chunks of 32 through shared
+// memory (stored transposed, k-major, with the next chunk's global loads
+// issued before the current chunk's FMAs); then top-k per token from the
+// logits, kept in the same shared memory.  fp32 FMAs in a fixed order.
+constexpr int RT_TOK = 128, RT_EXP = 64, RT_K = 32;
+constexpr int RT_XS = RT_TOK + 4, RT_WS = RT_EXP + 4;   // padded rows: conflict-free stores and loads
+
+struct RouteTiledSmem {
+    union {
+        struct {
+            float xs[RT_K][RT_XS];
+            float ws[RT_K][RT_WS];
+        } in;
+        float zs[RT_TOK][RT_EXP + 1];
+    };
+};
 
 __global__ void __launch_bounds__(256) route_tiled_kernel(const __nv_bfloat16* __restrict__ x,
                                                           const float* __restrict__ wr,
@@ -110,73 +123,97 @@ __global__ void __launch_bounds__(256) route_tiled_kernel(const __nv_bfloat16* _
                                                           int H, int E, int k, int renorm,
                                                           int32_t* __restrict__ idx,
                                                           float* __restrict__ w) {
-    __shared__ __align__(16) float xs[RT_K][RT_TOK + RT_PAD];
-    __shared__ __align__(16) float wsm[RT_K][RT_EXP + RT_PAD];
-    __shared__ float zs[RT_TOK][RT_EXP + 1];
+    __shared__ __align__(16) RouteTiledSmem sm;
     grid_dep_wait();
     grid_dep_launch();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.x * RT_TOK;
-    const int ty = tid >> 4, tx = tid & 15;
-    float acc[4][4];
+    const int ty = tid >> 4, tx = tid & 15;   // tokens ty*8.., experts tx*4..
+    float acc[8][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
-    const int lrow = tid >> 2;          // token (for x) / expert (for W) loaded by this thread
-    const int lseg = (tid & 3) * 8;     // 8 consecutive h
-    for (int h0 = 0; h0 < H; h0 += RT_K) {
-        {
-            const int t = t0 + lrow;
-            uint4 u = make_uint4(0, 0, 0, 0);
-            if (t < T)
-                u = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + h0 + lseg));
-            const uint32_t p[4] = {u.x, u.y, u.z, u.w};
+    // loader mapping: a warp covers 32 consecutive tokens (experts) of one
+    // 8-wide (4-wide) h segment, so the transposed stores hit 32 banks
+    const int xt = (tid & 31) + 32 * ((tid >> 5) >> 2);   // token 0..63 (+64 for the second load)
+    const int xseg = (tid >> 5) & 3;                       // 8 h each
+    const int we = tid & 63;                               // expert
+    const int wseg = tid >> 6;                             // 4 h each, 0..3 (+4 for the second load)
+    uint4 xr[2];
+    float4 wv[2];
+    auto fetch = [&](int h0) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int t = t0 + xt + 64 * i;
+            xr[i] = t < T ? __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + h0 + xseg * 8))
+                          : make_uint4(0, 0, 0, 0);
+            wv[i] = we < E ? __ldg(reinterpret_cast<const float4*>(wr + static_cast<size_t>(we) * H + h0 +
+                                                                    (wseg + 4 * i) * 4))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto stash = [&]() {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint32_t pq[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                xs[lseg + 2 * q][lrow] = __uint_as_float(p[q] << 16);
-                xs[lseg + 2 * q + 1][lrow] = __uint_as_float(p[q] & 0xffff0000u);
+                sm.in.xs[xseg * 8 + 2 * q][xt + 64 * i] = __uint_as_float(pq[q] << 16);
+                sm.in.xs[xseg * 8 + 2 * q + 1][xt + 64 * i] = __uint_as_float(pq[q] & 0xffff0000u);
             }
-            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-            if (lrow < E) {
-                const float4* src = reinterpret_cast<const float4*>(wr + static_cast<size_t>(lrow) * H + h0 + lseg);
-                a = __ldg(src);
-                b = __ldg(src + 1);
-            }
-            wsm[lseg + 0][lrow] = a.x; wsm[lseg + 1][lrow] = a.y;
-            wsm[lseg + 2][lrow] = a.z; wsm[lseg + 3][lrow] = a.w;
-            wsm[lseg + 4][lrow] = b.x; wsm[lseg + 5][lrow] = b.y;
-            wsm[lseg + 6][lrow] = b.z; wsm[lseg + 7][lrow] = b.w;
+            const int hb = (wseg + 4 * i) * 4;
+            sm.in.ws[hb + 0][we] = wv[i].x;
+            sm.in.ws[hb + 1][we] = wv[i].y;
+            sm.in.ws[hb + 2][we] = wv[i].z;
+            sm.in.ws[hb + 3][we] = wv[i].w;
         }
+    };
+    fetch(0);
+    for (int h0 = 0; h0 < H; h0 += RT_K) {
+        stash();
         __syncthreads();
-#pragma unroll 8
+        if (h0 + RT_K < H) fetch(h0 + RT_K);   // in flight during the FMAs below
+        // operands of step kk + 1 are read from shared memory while step kk's
+        // 32 FMAs run (few warps per SM: the load latency must hide in ILP)
+        float4 a0 = *reinterpret_cast<const float4*>(&sm.in.xs[0][ty * 8]);
+        float4 a1 = *reinterpret_cast<const float4*>(&sm.in.xs[0][ty * 8 + 4]);
+        float4 b = *reinterpret_cast<const float4*>(&sm.in.ws[0][tx * 4]);
+#pragma unroll
         for (int kk = 0; kk < RT_K; ++kk) {
-            const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
-            const float4 b = *reinterpret_cast<const float4*>(&wsm[kk][tx * 4]);
-            const float av[4] = {a.x, a.y, a.z, a.w};
+            float4 na0 = a0, na1 = a1, nb = b;
+            if (kk + 1 < RT_K) {
+                na0 = *reinterpret_cast<const float4*>(&sm.in.xs[kk + 1][ty * 8]);
+                na1 = *reinterpret_cast<const float4*>(&sm.in.xs[kk + 1][ty * 8 + 4]);
+                nb = *reinterpret_cast<const float4*>(&sm.in.ws[kk + 1][tx * 4]);
+            }
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+            a0 = na0;
+            a1 = na1;
+            b = nb;
         }
         __syncthreads();
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int t = t0 + ty * 4 + i, e = tx * 4 + j;
+            const int t = t0 + ty * 8 + i, e = tx * 4 + j;
             float zv = acc[i][j];
             if (bias && t < T && e < E) zv += __ldg(bias + static_cast<size_t>(t) * E + e);
-            zs[ty * 4 + i][e] = zv;
+            sm.zs[ty * 8 + i][e] = zv;
         }
     __syncthreads();
     for (int r = warp; r < RT_TOK; r += 8) {
         const int t = t0 + r;
         if (t >= T) break;
-        warp_topk_softmax(zs[r], E, k, renorm, idx + static_cast<size_t>(t) * k,
+        warp_topk_softmax(sm.zs[r], E, k, renorm, idx + static_cast<size_t>(t) * k,
                           w + static_cast<size_t>(t) * k, lane);
     }
 }
