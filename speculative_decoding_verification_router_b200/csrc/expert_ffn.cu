@@ -965,11 +965,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // flight; the first CTA issues one M = 256, N = 256 MMA per 16-wide k-slice
 // and each CTA's TMEM receives its 128 token rows x 256 columns.
 //   - both CTAs' loads complete on CTA 0's `full` barrier (armed by CTA 0
-//     for the pair's bytes), on which CTA 0's MMA thread waits; its commits
-//     arrive on `empty` (stage free) and `tfull` (accumulator ready) in both
-//     CTAs;
+//     for the pair's bytes), on which CTA 0's MMA thread waits; it commits
+//     each completion twice, to `empty` (stage free) and `tfull` (accumulator
+//     ready) of CTA 0 and of CTA 1, by cluster address;
 //   - both CTAs' epilogue warps arrive on CTA 0's `tempty` (count 8).
-// No TMA multicast: every load reads this GPU's memory into its own CTA.
+// No multicast of any kind: every load reads this GPU's memory into its own CTA.
 constexpr int PAIR_STAGE = 2 * TILE_BYTES;   // 128 token rows + 128 weight rows, 64 wide
 constexpr int PAIR_ST = 6;
 constexpr int PAIR_SMEM = PAIR_ST * PAIR_STAGE + 1024;
@@ -1093,6 +1093,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             Work w;
             // ---------------------------------------------------- MMA issuer (one thread of CTA 0)
             const uint32_t idesc = idesc_bf16_f32(2 * BM, 2 * BM);
+            // each completion is committed to this CTA's barrier and to the peer's
+            const uint32_t empty_self = mapa_shared(smem_addr(&bar_empty[0]), 0);
+            const uint32_t empty_peer = mapa_shared(smem_addr(&bar_empty[0]), 1);
+            const uint32_t tfull_self = mapa_shared(smem_addr(&bar_tfull[0]), 0);
+            const uint32_t tfull_peer = mapa_shared(smem_addr(&bar_tfull[0]), 1);
             int q = 0, acc = 0;
             uint32_t acc_phase = 0;
             while (ok && it.next(p, sched, w)) {
@@ -1113,10 +1118,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int kk = 0; kk < BK / 16; ++kk)
                         mma_bf16_pair(d0, smem_desc_sw128(a + kk * 32), smem_desc_sw128(b + kk * 32), idesc,
                                       (kt > w.k0 || kk > 0) ? 1u : 0u);
-                    mma_commit_pair(smem_addr(&bar_empty[stage]), 0x3);
+                    mma_commit_pair(empty_self + stage * 8);
+                    mma_commit_pair(empty_peer + stage * 8);
                 }
                 if (!ok) break;
-                mma_commit_pair(smem_addr(&bar_tfull[acc]), 0x3);
+                mma_commit_pair(tfull_self + acc * 8);
+                mma_commit_pair(tfull_peer + acc * 8);
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
             }
@@ -1126,7 +1133,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             tstamp(p, MODE, TS_LAST_MMA);
             // drain: every pair MMA issued by this thread completes before TMEM is freed
-            mma_commit_pair(smem_addr(&bar_drain), 0x1);
+            mma_commit_pair(mapa_shared(smem_addr(&bar_drain), 0));
             volatile int never = 0;
             if (!mbar_wait(smem_addr(&bar_drain), 0, lim, &never)) report_status(p.status, MS_ERR_TIMEOUT);
         }
