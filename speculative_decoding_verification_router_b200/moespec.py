@@ -132,6 +132,31 @@ def _ws(ws: Optional[Workspace], need: int, device) -> Workspace:
     return Workspace(max(need, 1), device)
 
 
+class CapturedStep:
+    """A fixed sequence of calls of this library (and the host<->device copies
+    around them) captured once into a CUDA graph and replayed as one launch,
+    for decode loops whose per-step host launch cost would otherwise exceed
+    the device time.  `fn` must use preallocated tensors and workspaces (the
+    graph replays the same addresses); it is run `warmup` times on `stream`
+    before capture.  Every library call launches its kernels on the current
+    stream, so the captured calls must not name another stream."""
+
+    def __init__(self, fn, stream=None, warmup: int = 2):
+        self.stream = stream or torch.cuda.Stream()
+        with torch.cuda.stream(self.stream):
+            for _ in range(warmup):
+                fn()
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            fn()
+        torch.cuda.synchronize()
+
+    def __call__(self):
+        with torch.cuda.stream(self.stream):
+            self.graph.replay()
+
+
 # ------------------------------------------------------------------ calls
 
 def pack_weights(w: torch.Tensor, stream=None) -> torch.Tensor:

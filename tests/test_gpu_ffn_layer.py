@@ -233,3 +233,28 @@ def test_trace_records_kernels(ms):
     assert names == ["route_cluster", "permute_scatter", "ffn_prep", "gemm1_stream", "ffn_finish", "gemm2_stream",
                      "ffn_finish", "combine"], names
     assert all(t > 0 for _, t in recs)
+
+
+def test_captured_step_replays_the_layer(ms):
+    # a layer call captured once (with its input copy) and replayed equals a direct call
+    shp = synth.VERIFY_B1
+    a, lw, bias = routed_layer_inputs(shp, 3)
+    wgu, wd, wsgu, wsd = _weights_dev(lw)
+    wr = dev(lw.w_router)
+    ws = ms.Workspace(ms.layer_workspace_size(shp.T, shp.H, shp.E, shp.I, shp.S, shp.k))
+    a_h = torch.from_numpy(a).pin_memory()
+    a_d = torch.empty_like(a_h, device="cuda")
+    out = torch.empty_like(a_d)
+
+    def fn():
+        a_d.copy_(a_h, non_blocking=True)
+        ms.layer_forward(a_d, wr, None, wgu, wd, wsgu, wsd, shp.k, ws=ws, out=out)
+
+    step = ms.CapturedStep(fn)
+    out.zero_()
+    step()
+    torch.cuda.synchronize()
+    got = out.clone()
+    direct = ms.layer_forward(dev(a), wr, None, wgu, wd, wsgu, wsd, shp.k)
+    torch.cuda.synchronize()
+    assert torch.equal(got, direct)
