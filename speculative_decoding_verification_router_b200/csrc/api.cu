@@ -22,7 +22,7 @@ size_t ffn_ws_bytes(int, int, int, int, int, int);
 ms_status ffn_launch(const void*, const int32_t*, const int32_t*, const void*, const void*, const void*,
                      const void*, int, int, int, int, int, int, void*, ms_dtype, float*, void*, cudaStream_t);
 ms_status combine_launch(const void*, ms_dtype, const float*, const int32_t*, const float*, const float*,
-                         int, int, int, float*, void*, cudaStream_t);
+                         int, int, int, float*, void*, cudaStream_t, bool);
 void set_device_trace(void*);
 
 static const char* kNames[K_COUNT] = {
@@ -175,7 +175,10 @@ ms_status moe_layer_forward(const float* a, const float* w_router, const float* 
         st = ms::ffn_launch(w.xhat, w.offsets, w.perm, w_gate_up, w_down, ws_gate_up, ws_down, T, H, E, I, S, k,
                             w.y_perm, ydt, S > 0 ? w.y_sh : nullptr, w.ffn_ws, s);
     if (st == MS_OK)
-        st = ms::combine_launch(w.y_perm, ydt, S > 0 ? w.y_sh : nullptr, w.slot, w.w, a, T, H, k, out, nullptr, s);
+        // slots and gate weights (router, permute) and the residual are several
+        // launches back: the combine may read them before its dependency wait
+        st = ms::combine_launch(w.y_perm, ydt, S > 0 ? w.y_sh : nullptr, w.slot, w.w, a, T, H, k, out, nullptr, s,
+                                true);
     return st;
 }
 

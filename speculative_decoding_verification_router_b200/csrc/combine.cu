@@ -22,6 +22,12 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
 }
 
 // One thread per 8 consecutive hidden elements of one token (grid-stride).
+// With `early` set (the layer's own chain, where the slots, gate weights and
+// residual were written two or more launches back), a thread reads those of
+// its first element before waiting on the previous kernel, leaving only the
+// expert outputs' round trip after the wait.
+constexpr int CB_KPRE = 8;
+
 template <typename TY>
 __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
                                                       const float* __restrict__ ysh,
@@ -29,25 +35,50 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
                                                       const float* __restrict__ w,
                                                       const float* __restrict__ res, int T, int H,
                                                       int k, float* __restrict__ out,
-                                                      __nv_bfloat16* __restrict__ out_bf16) {
-    grid_dep_wait();
-    grid_dep_launch();
+                                                      __nv_bfloat16* __restrict__ out_bf16, int early) {
     const int n8 = H >> 3;
     const long total = static_cast<long>(T) * n8;
     const long rows = static_cast<long>(T) * k;
-    for (long v = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; v < total;
-         v += static_cast<long>(gridDim.x) * blockDim.x) {
+    const long v0 = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x;
+    const bool pre = early && k <= CB_KPRE && v0 < total;
+    int pr[CB_KPRE];
+    float pw[CB_KPRE], prv[8];
+    if (pre) {
+        const int t = static_cast<int>(v0 / n8);
+#pragma unroll
+        for (int j = 0; j < CB_KPRE; ++j)
+            if (j < k) {
+                pr[j] = __ldg(slot + static_cast<size_t>(t) * k + j);
+                pw[j] = __ldg(w + static_cast<size_t>(t) * k + j);
+            }
+        if (res) load8(res + static_cast<size_t>(t) * H + static_cast<int>(v0 % n8) * 8, prv);
+    }
+    grid_dep_wait();
+    grid_dep_launch();
+    for (long v = v0; v < total; v += static_cast<long>(gridDim.x) * blockDim.x) {
         const int t = static_cast<int>(v / n8);
         const int c = static_cast<int>(v % n8) * 8;
+        const bool first = pre && v == v0;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < k; ++j) {
-            const int r = __ldg(slot + static_cast<size_t>(t) * k + j);
-            if (r < 0 || r >= rows) continue;
-            const float wj = __ldg(w + static_cast<size_t>(t) * k + j);
-            float yv[8];
-            load8(y + static_cast<size_t>(r) * H + c, yv);
+        if (first) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) acc[q] = fmaf(wj, yv[q], acc[q]);
+            for (int j = 0; j < CB_KPRE; ++j) {
+                if (j >= k || pr[j] < 0 || pr[j] >= rows) continue;
+                float yv[8];
+                load8(y + static_cast<size_t>(pr[j]) * H + c, yv);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] = fmaf(pw[j], yv[q], acc[q]);
+            }
+        } else {
+            for (int j = 0; j < k; ++j) {
+                const int r = __ldg(slot + static_cast<size_t>(t) * k + j);
+                if (r < 0 || r >= rows) continue;
+                const float wj = __ldg(w + static_cast<size_t>(t) * k + j);
+                float yv[8];
+                load8(y + static_cast<size_t>(r) * H + c, yv);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] = fmaf(wj, yv[q], acc[q]);
+            }
         }
         const size_t o = static_cast<size_t>(t) * H + c;
         if (ysh) {
@@ -58,7 +89,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
         }
         if (res) {
             float rv[8];
-            load8(res + o, rv);
+            if (first) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) rv[q] = prv[q];
+            } else {
+                load8(res + o, rv);
+            }
 #pragma unroll
             for (int q = 0; q < 8; ++q) acc[q] += rv[q];
         }
@@ -76,16 +112,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const TY* __restrict__ y,
 
 ms_status combine_launch(const void* y, ms_dtype ydt, const float* ysh, const int32_t* slot,
                          const float* w, const float* res, int T, int H, int k, float* out,
-                         void* out_bf16, cudaStream_t s) {
+                         void* out_bf16, cudaStream_t s, bool early) {
     const long total = static_cast<long>(T) * (H / 8);
     const long want = (total + 255) / 256;
     const int grid = static_cast<int>(want < 8L * num_sms() ? want : 8L * num_sms());
     auto* ob = reinterpret_cast<__nv_bfloat16*>(out_bf16);
     if (ydt == MS_BF16)
         return launch(K_COMBINE, combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s,
-                      reinterpret_cast<const __nv_bfloat16*>(y), ysh, slot, w, res, T, H, k, out, ob);
+                      reinterpret_cast<const __nv_bfloat16*>(y), ysh, slot, w, res, T, H, k, out, ob, early ? 1 : 0);
     return launch(K_COMBINE, combine_kernel<float>, dim3(grid), dim3(256), 0, s,
-                  reinterpret_cast<const float*>(y), ysh, slot, w, res, T, H, k, out, ob);
+                  reinterpret_cast<const float*>(y), ysh, slot, w, res, T, H, k, out, ob, early ? 1 : 0);
 }
 
 }  // namespace ms
@@ -102,5 +138,5 @@ extern "C" ms_status moe_combine(const void* y_perm, ms_dtype y_perm_dtype, cons
         (residual && !ms::aligned16(residual)) || (out_bf16 && !ms::aligned16(out_bf16)))
         return MS_ERR_INVALID_ARG;
     return ms::combine_launch(y_perm, y_perm_dtype, y_shared, slot_of, topk_w, residual, T, H, k,
-                              out, out_bf16, static_cast<cudaStream_t>(stream));
+                              out, out_bf16, static_cast<cudaStream_t>(stream), false);
 }

@@ -111,7 +111,7 @@ ms_status linear_launch(const void*, int, int, int, const void*, int, const int3
                         cudaStream_t);
 ms_status rmsnorm_launch(const float*, const float*, int, int, float, void*, cudaStream_t);
 ms_status combine_launch(const void*, ms_dtype, const float*, const int32_t*, const float*, const float*, int,
-                         int, int, float*, void*, cudaStream_t);
+                         int, int, float*, void*, cudaStream_t, bool);
 ms_status verify_keys_launch(const unsigned long long*, int, int, int, const int32_t*, int32_t*, int32_t*,
                              int32_t*, cudaStream_t);
 
@@ -204,7 +204,7 @@ extern "C" ms_status fastmtp_draft(const float* h0, const int32_t* tok0, const v
             st = ms::ffn_launch(w.xh, w.offsets, w.perm, w_gate_up, w_down, nullptr, nullptr, B, H, 1, I, 0, 1, w.y,
                                 MS_F32, nullptr, w.ffn, s);
         if (st == MS_OK)
-            st = ms::combine_launch(w.y, MS_F32, nullptr, w.slot, w.w1, w.u, B, H, 1, h_next, nullptr, s);
+            st = ms::combine_launch(w.y, MS_F32, nullptr, w.slot, w.w1, w.u, B, H, 1, h_next, nullptr, s, false);
         if (st == MS_OK) st = ms::rmsnorm_launch(h_next, nullptr, B, H, eps, w.xh, s);
         if (st == MS_OK) st = ms::lm_launch(w.xh, w_lm, B, H, V, nullptr, w.lm, s, w.keys, status);
         if (st == MS_OK)

@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(256) route_tiled_kernel(const __nv_bfloat16* _
 // row themselves (eps, unit gain) and CTA 0 writes the bf16 result, so the
 // layer needs no separate normalisation kernel.
 constexpr int RC_CTAS = 8;
+constexpr int RC_WPRE = 12;   // float4 of a router row per lane kept in registers (H <= 1536)
 
 template <bool NORM>
 __global__ void __launch_bounds__(256) route_cluster_kernel(const void* __restrict__ xin,
@@ -243,6 +244,21 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(const void* __restri
     const uint32_t rank = cluster_rank();
     const int t = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int per = (E + RC_CTAS - 1) / RC_CTAS;
+    const int e0 = static_cast<int>(rank) * per;
+    const int e1 = e0 + per < E ? e0 + per : E;
+    // this warp's first router row, loaded together with the activation row
+    // (independent loads, one round trip) when it fits the registers
+    const bool wpre = H / 4 <= 32 * RC_WPRE && e0 + warp < e1;
+    float4 wv[RC_WPRE];
+    if (wpre) {
+        const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(e0 + warp) * H);
+#pragma unroll
+        for (int j = 0; j < RC_WPRE; ++j) {
+            const int h4 = lane + 32 * j;
+            wv[j] = h4 < H / 4 ? __ldg(wrow + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
     if (NORM) {
         const float4* row = reinterpret_cast<const float4*>(static_cast<const float*>(xin) + static_cast<size_t>(t) * H);
         float ss = 0.f;
@@ -284,20 +300,31 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(const void* __restri
         }
     }
     __syncthreads();
-    const int per = (E + RC_CTAS - 1) / RC_CTAS;
-    const int e0 = static_cast<int>(rank) * per;
-    const int e1 = e0 + per < E ? e0 + per : E;
     for (int e = e0 + warp; e < e1; e += 8) {
         const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * H);
         float acc = 0.f;
+        if (wpre && e == e0 + warp) {
+#pragma unroll
+            for (int j = 0; j < RC_WPRE; ++j) {
+                const int h4 = lane + 32 * j;
+                if (h4 < H / 4) {
+                    const float4 b = *reinterpret_cast<const float4*>(xs + 4 * h4);
+                    acc = fmaf(wv[j].x, b.x, acc);
+                    acc = fmaf(wv[j].y, b.y, acc);
+                    acc = fmaf(wv[j].z, b.z, acc);
+                    acc = fmaf(wv[j].w, b.w, acc);
+                }
+            }
+        } else {
 #pragma unroll 4
-        for (int h4 = lane; h4 < H / 4; h4 += 32) {
-            const float4 a = __ldg(wrow + h4);
-            const float4 b = *reinterpret_cast<const float4*>(xs + 4 * h4);
-            acc = fmaf(a.x, b.x, acc);
-            acc = fmaf(a.y, b.y, acc);
-            acc = fmaf(a.z, b.z, acc);
-            acc = fmaf(a.w, b.w, acc);
+            for (int h4 = lane; h4 < H / 4; h4 += 32) {
+                const float4 a = __ldg(wrow + h4);
+                const float4 b = *reinterpret_cast<const float4*>(xs + 4 * h4);
+                acc = fmaf(a.x, b.x, acc);
+                acc = fmaf(a.y, b.y, acc);
+                acc = fmaf(a.z, b.z, acc);
+                acc = fmaf(a.w, b.w, acc);
+            }
         }
         acc = warp_sum(acc);
         if (lane == 0) st_cluster_f32(&z[e], 0, bias ? acc + __ldg(bias + static_cast<size_t>(t) * E + e) : acc);

@@ -203,9 +203,10 @@ ms_status verify_keys_launch(const unsigned long long* keys, int ld, int B, int 
 // CTA 0 merges the P chunks of each row and runs the prefix match.
 constexpr int VC_THREADS = 512;
 constexpr int VC_MAX = 16;
-constexpr int VC_UNROLL = 4;
 
-template <typename TL>
+// UNROLL: 16-byte loads in flight per thread -- 8 for small batches (latency:
+// one round trip for a 64 KB chunk), 4 for large ones (occupancy).
+template <typename TL, int UNROLL>
 __global__ void __launch_bounds__(VC_THREADS) verify_cluster_kernel(const TL* __restrict__ logits, int K, int V,
                                                                     int P, int chunk, int vec_ok,
                                                                     const int32_t* __restrict__ draft,
@@ -232,15 +233,15 @@ __global__ void __launch_bounds__(VC_THREADS) verify_cluster_kernel(const TL* __
         int tail_begin = begin;
         if (vec_ok && end > begin) {
             const int nvec = (end - begin) / VEC;
-            for (int q0 = threadIdx.x; q0 < nvec; q0 += VC_UNROLL * VC_THREADS) {
-                float v[VC_UNROLL][VEC];
+            for (int q0 = threadIdx.x; q0 < nvec; q0 += UNROLL * VC_THREADS) {
+                float v[UNROLL][VEC];
 #pragma unroll
-                for (int u = 0; u < VC_UNROLL; ++u) {
+                for (int u = 0; u < UNROLL; ++u) {
                     const int q = q0 + u * VC_THREADS;
                     if (q < nvec) vec_load(row + begin + q * VEC, v[u]);
                 }
 #pragma unroll
-                for (int u = 0; u < VC_UNROLL; ++u) {
+                for (int u = 0; u < UNROLL; ++u) {
                     const int q = q0 + u * VC_THREADS;
                     if (q < nvec) {
 #pragma unroll
@@ -298,15 +299,19 @@ __global__ void __launch_bounds__(VC_THREADS) verify_cluster_kernel(const TL* __
     }
 }
 
+template <typename TL, int U>
+static bool allow_big_clusters() {
+    return cudaFuncSetAttribute(verify_cluster_kernel<TL, U>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+           cudaSuccess;
+}
+
 static int verify_cluster_size() {
     // 16-CTA clusters when the device allows them, else the portable 8
     static int cs = 0;
     if (cs == 0) {
         cs = 8;
-        if (cudaFuncSetAttribute(verify_cluster_kernel<__nv_bfloat16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-                cudaSuccess &&
-            cudaFuncSetAttribute(verify_cluster_kernel<float>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-                cudaSuccess) {
+        if (allow_big_clusters<__nv_bfloat16, 4>() && allow_big_clusters<__nv_bfloat16, 8>() &&
+            allow_big_clusters<float, 4>() && allow_big_clusters<float, 8>()) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(16, 1);
             cfg.blockDim = dim3(VC_THREADS);
@@ -318,7 +323,8 @@ static int verify_cluster_size() {
             cfg.attrs = at;
             cfg.numAttrs = 1;
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, verify_cluster_kernel<__nv_bfloat16>, &cfg) == cudaSuccess && n > 0)
+            if (cudaOccupancyMaxActiveClusters(&n, verify_cluster_kernel<__nv_bfloat16, 8>, &cfg) == cudaSuccess &&
+                n > 0)
                 cs = 16;
         }
         cudaGetLastError();
@@ -340,13 +346,21 @@ static ms_status verify_cluster_launch(const void* logits, ms_dtype dt, const in
     P = (V + chunk - 1) / chunk;
     const int cs = (K + 1) * P;
     const int vec_ok = (V % vec == 0) && aligned16(logits);
+    // one CTA per SM at most: unroll for latency; more CTAs than SMs: for occupancy
+    const bool few = static_cast<long>(cs) * B <= num_sms();
+    const __nv_bfloat16* lb = reinterpret_cast<const __nv_bfloat16*>(logits);
+    const float* lf = reinterpret_cast<const float*>(logits);
     if (dt == MS_BF16)
-        return launch_cluster(K_VERIFY_CLUSTER, verify_cluster_kernel<__nv_bfloat16>, dim3(cs, B), dim3(VC_THREADS), 0,
-                              s, cs, reinterpret_cast<const __nv_bfloat16*>(logits), K, V, P, chunk, vec_ok, draft,
-                              argmax, committed, ncom);
-    return launch_cluster(K_VERIFY_CLUSTER, verify_cluster_kernel<float>, dim3(cs, B), dim3(VC_THREADS), 0, s, cs,
-                          reinterpret_cast<const float*>(logits), K, V, P, chunk, vec_ok, draft, argmax, committed,
-                          ncom);
+        return few ? launch_cluster(K_VERIFY_CLUSTER, verify_cluster_kernel<__nv_bfloat16, 8>, dim3(cs, B),
+                                    dim3(VC_THREADS), 0, s, cs, lb, K, V, P, chunk, vec_ok, draft, argmax, committed,
+                                    ncom)
+                   : launch_cluster(K_VERIFY_CLUSTER, verify_cluster_kernel<__nv_bfloat16, 4>, dim3(cs, B),
+                                    dim3(VC_THREADS), 0, s, cs, lb, K, V, P, chunk, vec_ok, draft, argmax, committed,
+                                    ncom);
+    return few ? launch_cluster(K_VERIFY_CLUSTER, verify_cluster_kernel<float, 8>, dim3(cs, B), dim3(VC_THREADS), 0,
+                                s, cs, lf, K, V, P, chunk, vec_ok, draft, argmax, committed, ncom)
+               : launch_cluster(K_VERIFY_CLUSTER, verify_cluster_kernel<float, 4>, dim3(cs, B), dim3(VC_THREADS), 0,
+                                s, cs, lf, K, V, P, chunk, vec_ok, draft, argmax, committed, ncom);
 }
 
 struct VerifyPlan {
