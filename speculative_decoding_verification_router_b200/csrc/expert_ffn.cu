@@ -10,17 +10,20 @@
 // Two schedules:
 //  * streaming (verify-sized T <= 128): the weights are the M = 128 operand
 //    and the tokens of one expert the N operand (N = rows rounded up to 16).
-//    The work -- every (group, 128-feature tile, 64-wide k-step) -- is
-//    divided into equal contiguous ranges of k-steps, one per CTA, so every
-//    SM streams the same number of weight bytes ("stream-K").  A tile split
-//    between CTAs is finished by the last CTA to arrive, which sums the fp32
-//    partials in CTA order (deterministic, no waiting on other CTAs).
+//    Every CTA takes the same number of whole output tiles, all but the last
+//    round; the k-steps of the remaining tiles are divided into equal
+//    contiguous ranges, one per CTA, so every SM streams the same number of
+//    weight bytes ("stream-K").  A CTA's part of a split tile goes to an fp32
+//    partial slot; ffn_finish_kernel, launched after the GEMM, sums the two
+//    or three parts of each split tile in CTA order (deterministic, no CTA
+//    ever waits on another) and applies the epilogue.
 //    For GEMM1 the gate and up rows of the same 128 features accumulate into
 //    two TMEM buffers in the same lanes, so SwiGLU is done in registers.
 //  * tiled (prefill-sized T): the tokens of one expert are the M = 128
 //    operand and the weights the N operand; for GEMM1 the N = 256 tile is
 //    128 gate rows followed by the matching 128 up rows, so each thread holds
-//    both halves of its token row and applies SwiGLU in registers.
+//    both halves of its token row and applies SwiGLU in registers.  GEMM2
+//    runs 256 x 256 tiles on CTA pairs (ffn_gemm_pair_kernel).
 // Shared experts form one extra group whose intermediate width is S*I: two
 // SwiGLU experts equal one expert with the intermediates concatenated.
 #include <cuda.h>
