@@ -64,6 +64,16 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert fused(fake, fake, fake, 2, 3, 256, 1024, fake, fake, fake, None, 0, None) == -3         # no ws
     assert lib.spec_verify_lm_head_workspace_size(32, 3, 1280, 129280) > 32 * 4 * 8
     assert lib.spec_verify_lm_head_workspace_size(0, 3, 1280, 129280) == 0
+    # empty inputs are rejected before any launch
+    lib.moe_permute.restype = I
+    lib.moe_permute.argtypes = [P, I, I, I, P, P, P, P, Z, P]
+    assert lib.moe_permute(fake, 0, 6, 64, fake, fake, fake, None, 0, None) == -1              # T = 0
+    lib.moe_layer_forward.restype = I
+    lib.moe_layer_forward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, Z, P]
+    assert lib.moe_layer_forward(fake, fake, None, fake, fake, fake, fake, 0, 1280, 64, 896, 2, 6, 0, fake, fake,
+                                 1 << 30, None) == -1                                          # T = 0
+    assert lib.spec_verify_greedy(fake, 1, fake, 0, 3, 100, fake, fake, fake, fake, 1 << 20, None) == -1  # B = 0
+    assert lib.spec_verify_greedy(fake, 1, None, 2, 0, 100, fake, fake, fake, None, 0, None) == -3  # K = 0 needs no drafts
     lib.moe_expert_ffn_workspace_size.restype = ctypes.c_size_t
     lib.moe_expert_ffn_workspace_size.argtypes = [I] * 6
     assert lib.moe_expert_ffn_workspace_size(4, 1280, 64, 896, 2, 6) > 0

@@ -258,3 +258,29 @@ def test_captured_step_replays_the_layer(ms):
     direct = ms.layer_forward(dev(a), wr, None, wgu, wd, wsgu, wsd, shp.k)
     torch.cuda.synchronize()
     assert torch.equal(got, direct)
+
+
+DEGENERATE = [
+    synth.MoEShape("all_experts_k_eq_E", B=4, K=3, H=256, E=8, I=128, k=8, S=1, V=1024, router_std=0.05),
+    synth.MoEShape("no_shared_expert", B=4, K=3, H=256, E=8, I=128, k=2, S=0, V=1024, router_std=0.05),
+    synth.MoEShape("dense_one_expert", B=4, K=3, H=256, E=1, I=256, k=1, S=0, V=1024, router_std=0.05),
+    synth.MoEShape("single_token", B=1, K=0, H=256, E=8, I=128, k=2, S=1, V=1024, router_std=0.05, tokens=1),
+    synth.MoEShape("max_streaming_tokens", B=1, K=0, H=256, E=16, I=128, k=4, S=1, V=1024, router_std=0.05,
+                   tokens=128),
+]
+
+
+@pytest.mark.parametrize("shp", DEGENERATE, ids=[w.name for w in DEGENERATE])
+def test_layer_degenerate_shapes(ms, shp):
+    # every expert chosen (k = E), no shared expert, a dense layer (E = 1), a
+    # single token, and the largest batch of the streaming schedule
+    a, lw, bias = routed_layer_inputs(shp, 0)
+    ref = oracle.moe_layer(a, lw, shp.k, bias)
+    wgu, wd, wsgu, wsd = _weights_dev(lw)
+    ws = ms.Workspace(ms.layer_workspace_size(shp.T, shp.H, shp.E, shp.I, shp.S, shp.k))
+    out = ms.layer_forward(dev(a), dev(lw.w_router), None if bias is None else dev(bias), wgu, wd, wsgu, wsd,
+                           shp.k, ws=ws)
+    assert ms.device_status(ws) == 0
+    o = host(out)
+    assert_close(o, ref["out"], what="out")
+    assert_close(o - a, ref["out"] - a, what="moe delta")
