@@ -208,11 +208,16 @@ class Problem:
         s = self.shp
         self.ms.layer_forward(a, L["wr"], self.bias, L["wgu"], L["wd"], L["wsgu"], L["wsd"], s.k, ws=self.ws, out=out)
 
-    def step(self, i: int):
+    def step(self, i: int, before_verify=None):
+        """One step.  `before_verify`, if given, runs on the host just before the
+        verify launch (the end-to-end path makes the stream wait there for the
+        drafts and logits it copies on a second stream)."""
         s = self.shp
         if s.layers == 1:
             self.layer(i, self.a, self.out)
             if self.verify:
+                if before_verify:
+                    before_verify()
                 self.ms.verify_greedy(self.logits[i % self.n_logit_sets], self.draft, ws=self.vws, out=self.vout)
             return
         # 12-layer decode step: h_l = h_{l-1} + a + MoE(RMSNorm(h_{l-1} + a)); the
@@ -223,6 +228,8 @@ class Problem:
             self.layer(l, cur, nxt)
             cur = nxt
         self.ms.rmsnorm(cur, out=self.xn)
+        if before_verify:
+            before_verify()
         if self.fused_head:
             # vocab head with the argmax in its epilogue, then the prefix match
             self.ms.verify_lm_head_greedy(self.xn, self.lm, self.draft, ws=self.fws, out=self.vout)
@@ -378,7 +385,7 @@ def run_ours(args, rank, world, local):
                     "peak_source": peaks["source"]}
 
     # end to end through the public API with host buffers
-    e2e = run_e2e(prob, ms, stream, steps=min(steps, 2000), world=world, device=device)
+    e2e = run_e2e(prob, ms, stream, steps=min(steps, 2000), world=world, device=device, direct=args.e2e_direct)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "verified tokens/s", "n_gpus": world,
@@ -424,7 +431,7 @@ def routed_work(prob, ms, stream):
     return {key: float(np.mean(v)) for key, v in acc.items()}
 
 
-def run_e2e(prob, ms, stream, steps, world, device):
+def run_e2e(prob, ms, stream, steps, world, device, direct=False):
     """Same step through the public API with pinned host inputs/outputs per step."""
     import torch
     shp = prob.shp
@@ -445,21 +452,37 @@ def run_e2e(prob, ms, stream, steps, world, device):
             h2d += lg_h.numel() * 2
         else:
             lg_h = None
+    # The verify inputs (drafts, and the logits when they come from the host)
+    # are needed only after the layer: they are copied on a second stream while
+    # the layer runs, and the verify launch waits for that copy.
+    copy_stream = torch.cuda.Stream(device=device)
+
+    def one_step(i):
+        cur = torch.cuda.current_stream()
+        prob.a.copy_(a_h, non_blocking=True)
+        if prob.verify:
+            copy_stream.wait_stream(cur)   # ordered after this step's start (the previous verify is done)
+            with torch.cuda.stream(copy_stream):
+                prob.draft.copy_(d_h, non_blocking=True)
+                if lg_h is not None:
+                    prob.logits[i % prob.n_logit_sets].copy_(lg_h, non_blocking=True)
+        prob.step(i, before_verify=(lambda: cur.wait_stream(copy_stream)) if prob.verify else None)
+        out_h.copy_(prob.out if shp.layers == 1 else prob.h[(shp.layers - 1) % 2], non_blocking=True)
+        if prob.verify:
+            n_h.copy_(prob.vout[2], non_blocking=True)
+            c_h.copy_(prob.vout[1], non_blocking=True)
+
+    # One captured step per weight set (the steps rotate over the sets as in
+    # the device-timed run): each replay is one launch of the whole step,
+    # copies included.  direct=True issues the library calls one by one.
+    steps_fn = ([(lambda i=i: one_step(i)) for i in range(prob.n_sets)] if direct else
+                [ms.CapturedStep(lambda i=i: one_step(i), stream=stream) for i in range(prob.n_sets)])
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         for i in range(steps + 3):
             if i == 3:
                 ev0.record(stream)
-            prob.a.copy_(a_h, non_blocking=True)
-            if prob.verify:
-                prob.draft.copy_(d_h, non_blocking=True)
-                if lg_h is not None:
-                    prob.logits[i % prob.n_logit_sets].copy_(lg_h, non_blocking=True)
-            prob.step(i)
-            out_h.copy_(prob.out if shp.layers == 1 else prob.h[(shp.layers - 1) % 2], non_blocking=True)
-            if prob.verify:
-                n_h.copy_(prob.vout[2], non_blocking=True)
-                c_h.copy_(prob.vout[1], non_blocking=True)
+            steps_fn[i % len(steps_fn)]()
             stream.synchronize()    # the caller needs the committed tokens before the next step
         ev1.record(stream)
     torch.cuda.synchronize()
@@ -467,7 +490,9 @@ def run_e2e(prob, ms, stream, steps, world, device):
     value = aggregate_rate(shp.T * steps, world, ms_total / 1e3)
     return {"value": round(value, 1), "unit": "verified tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms_total / steps, 5),
-            "sync": "stream synchronize after every step"}
+            "sync": "stream synchronize after every step",
+            "launch": "library calls one by one" if direct else "one CUDA graph launch per step (CapturedStep)",
+            "copies": "layer input on the compute stream; drafts and logits on a second stream, overlapped with the layer"}
 
 
 # ------------------------------------------------------------------ oracle (CPU)
@@ -674,6 +699,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=0, help="prefill workload: token count (a smaller case to profile)")
     ap.add_argument("--k-sweep", action="store_true",
                     help="12-layer step at B=32 for K = 0..3: step time, tau, spec-step cost and speedup")
+    ap.add_argument("--e2e-direct", action="store_true",
+                    help="end-to-end leg: library calls one by one instead of one captured graph per step")
     ap.add_argument("--fused-head", action="store_true",
                     help="12-layer step: argmax in the vocab head's epilogue (spec_verify_lm_head_greedy) "
                          "instead of writing the logits and verifying them in a separate kernel")

@@ -43,6 +43,7 @@ constexpr int TILE_BYTES = BM * BK * 2;  // 16 KB: 128 rows x 64 bf16
 constexpr int TOKBOX = 16;               // token rows per TMA box (streaming)
 constexpr int NTHREADS = 192;
 constexpr int MAX_GROUPS = 257;
+constexpr int MAX_CTAS = 256;            // streaming grid (one CTA per SM)
 constexpr int TMEM_COLS = 512;
 #ifndef MS_WEIGHT_BUDGET_KB
 #define MS_WEIGHT_BUDGET_KB 128
@@ -78,6 +79,7 @@ struct Params {
     unsigned long long* amax_key;  // vocab head, fused argmax: [T][V/16] keys instead of logits (NMAX 128)
     float* partials;               // 2 partial-sum slots per CTA (streaming)
     int nct;                       // grid size of the streaming GEMM (for the finish kernel)
+    int weights_evict_first;       // streaming: weight tiles are loaded with an L2 evict-first policy
     int32_t* status;
     uint64_t wait_limit_ns;
     uint64_t* dtrace;              // optional per-CTA timeline (see ms_set_device_trace)
@@ -123,6 +125,12 @@ struct Sched {
     int tprefix[MAX_GROUPS + 1];  // streaming: output tiles before group g
     int rows[MAX_GROUPS];
     int row0[MAX_GROUPS];
+    // streaming: the split region is the k-steps [sk_begin, total); cpre[g] is
+    // the cost (step_cost units) of its k-steps that lie before group g, and
+    // CTA c's split range is the k-steps [rb[c], rb[c + 1])
+    int sk_begin;
+    int cpre[MAX_GROUPS + 1];
+    int rb[MAX_CTAS + 1];
 };
 
 // Inclusive-to-exclusive scan of a[1..n] in place (a[0] = 0), by one warp.
@@ -152,6 +160,16 @@ __device__ __forceinline__ void warp_scan_groups(int* a, int n, int lane) {
     if (lane == 0) a[0] = 0;
 }
 
+// largest g with tprefix[g] <= t
+__device__ __forceinline__ int find_group_tile(const Sched& s, int t) {
+    int lo = 0, hi = s.ngroups - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s.tprefix[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
 template <int MODE>
 __device__ __forceinline__ int group_ktiles(const Params& p, int g) {
     const bool shared = p.offsets != nullptr && g == p.E;
@@ -167,6 +185,29 @@ __device__ __forceinline__ int group_ntiles(const Params& p, int g) {
     if (MODE == G1_STREAM || MODE == G1_TILED) return (shared ? p.S * p.I : p.I) / BM;
     if (MODE == G2_STREAM) return p.H / BM;
     return p.H / p.bn;   // G2_TILED
+}
+
+// Whole tiles per CTA on the streaming schedule: every full round of tiles
+// but the last, so that the split region holds the last nct .. 2 nct - 1
+// tiles (all of them when NT < nct).  Each CTA's split range is then about
+// one tile long, and a split tile has two or three contributors (four for
+// the costliest tiles), which the finish kernel sums in one or two rounds of
+// loads.
+__device__ __forceinline__ int dp_tiles_per_cta(int nt, int nct) {
+    const int q = nt / nct;
+    return q > 0 ? q - 1 : 0;
+}
+
+// Cost of one k-step of group g on the streaming schedule, in 2 KB units of
+// data the CTA moves: the weight tiles (32 KB) and the group's token boxes
+// (2 KB per 16 rows and 64-wide k-block).  The token boxes come from L2, but
+// a CTA's loads progress at its share of the memory system whatever their
+// source, so the split ranges are cut at equal cost rather than at equal
+// k-steps: a range over the shared experts' 128-token group holds fewer
+// k-steps than one over a 12-token expert.
+template <int MODE>
+__device__ __forceinline__ int step_cost(const Sched& s, int g) {
+    return 16 + Cfg<MODE>::kSub * ((s.rows[g] + TOKBOX - 1) / TOKBOX);
 }
 
 template <int MODE, int NT>
@@ -211,6 +252,57 @@ __device__ void build_schedule_n(const Params& p, Sched& s) {
     if (tid < 32) warp_scan_groups(s.prefix, ng, tid);
     else if (tid < 64) warp_scan_groups(s.tprefix, ng, tid - 32);
     __syncthreads();
+    if (Cfg<MODE>::kStream) {
+        // the split region: the tiles after the nct * D whole tiles
+        if (tid == 0) {
+            const int nt = s.tprefix[ng];
+            const int fs = p.nct * dp_tiles_per_cta(nt, p.nct);
+            int skb = s.prefix[ng];
+            if (fs < nt) {
+                const int g = find_group_tile(s, fs);
+                skb = s.prefix[g] + (fs - s.tprefix[g]) * group_ktiles<MODE>(p, g);
+            }
+            s.sk_begin = skb;
+        }
+        __syncthreads();
+        for (int g = tid; g < ng; g += NT) {
+            const int lo = max(s.prefix[g], s.sk_begin), hi = s.prefix[g + 1];
+            s.cpre[g + 1] = hi > lo ? (hi - lo) * step_cost<MODE>(s, g) : 0;
+        }
+        __syncthreads();
+        if (tid < 32) warp_scan_groups(s.cpre, ng, tid);
+        __syncthreads();
+        // CTA c's range starts at the first k-step whose cost prefix reaches
+        // c/nct of the region's cost
+        const int nct = p.nct, total = s.prefix[ng];
+        const long long C = s.cpre[ng];
+        // 32-bit arithmetic when the scaled costs fit (every layer of this
+        // model); 64-bit division is several times slower
+        const bool narrow = C * nct < (1LL << 31);
+        for (int c = tid; c <= nct; c += NT) {
+            int b;
+            if (c == 0 || C == 0) {
+                b = s.sk_begin;
+            } else if (c == nct) {
+                b = total;
+            } else {
+                const long long x = C * c;   // the target cost, times nct
+                int lo = 0, hi = ng - 1;     // largest g with cpre[g] * nct <= x
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (static_cast<long long>(s.cpre[mid]) * nct <= x) lo = mid; else hi = mid - 1;
+                }
+                const long long num = x - static_cast<long long>(s.cpre[lo]) * nct;
+                const long long den = static_cast<long long>(nct) * step_cost<MODE>(s, lo);
+                const int d = narrow ? static_cast<int>((static_cast<uint32_t>(num) + static_cast<uint32_t>(den) - 1u) /
+                                                        static_cast<uint32_t>(den))
+                                     : static_cast<int>((num + den - 1) / den);
+                b = max(s.prefix[lo], s.sk_begin) + d;
+            }
+            s.rb[c] = b;
+        }
+        __syncthreads();
+    }
 }
 
 template <int MODE>
@@ -230,15 +322,6 @@ __device__ __forceinline__ int find_group(const Sched& s, int pos) {
 struct Seg {
     int g, tile, k0, k1, kt, tile_start;   // tile: n-tile (streaming) / linear tile in group (tiled)
 };
-
-__device__ __forceinline__ long range_begin(int c, int total, int nct) {
-    return static_cast<long>(c) * total / nct;
-}
-// CTA whose range holds step `pos`: largest c with floor(c*total/nct) <= pos.
-__device__ __forceinline__ int cta_of(int pos, int total, int nct) {
-    const long num = static_cast<long>(pos + 1) * nct;
-    return static_cast<int>((num + total - 1) / total) - 1;
-}
 
 template <int MODE>
 __device__ __forceinline__ Seg stream_seg(const Params& p, const Sched& s, int pos, int end) {
@@ -268,25 +351,7 @@ struct Work {
 // once; partial tiles keep their natural order.
 __device__ __forceinline__ int kstep_of(const Work& w, int i) { return w.rot ? (i + w.rot) % w.kt : i; }
 
-// largest g with tprefix[g] <= t
-__device__ __forceinline__ int find_group_tile(const Sched& s, int t) {
-    int lo = 0, hi = s.ngroups - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s.tprefix[mid] <= t) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
 
-// Whole tiles per CTA on the streaming schedule: every full round of tiles
-// but the last, so that the split region holds the last nct .. 2 nct - 1
-// tiles (all of them when NT < nct).  Each CTA's split range is then at least
-// one tile long and a split tile has two contributors, three at most, so the
-// finish kernel sums it in one round of loads.
-__device__ __forceinline__ int dp_tiles_per_cta(int nt, int nct) {
-    const int q = nt / nct;
-    return q > 0 ? q - 1 : 0;
-}
 
 template <int MODE>
 struct WorkIter {
@@ -294,30 +359,24 @@ struct WorkIter {
     // tiles in group order and nct CTAs, CTA c owns the D = dp_tiles_per_cta
     // whole tiles [c*D, c*D + D); the k-steps of the remaining NT - nct*D
     // tiles at the end of the order (the split region) are divided into nct
-    // equal ranges.  A CTA walks its split range first and its whole tiles
-    // last.  Contributors to a split tile store fp32 partials; the finish
-    // kernel that follows the GEMM sums them and applies the epilogue.
+    // ranges of equal cost (step_cost).  A CTA walks its split range first
+    // and its whole tiles last.  Contributors to a split tile store fp32
+    // partials; the finish kernel that follows the GEMM sums them and applies
+    // the epilogue.
     // Tiled: tiles c, c + nct, ... (round robin).
     int c, nct, state, pos, re, dp_next, dp_end, t, total;
-    int sk_begin, sk_total;   // split region in absolute k-step positions
+    const Sched* sp;
 
     __device__ void init(const Params& p, const Sched& s, int c_, int nct_) {
         c = c_;
         nct = nct_;
+        sp = &s;
         total = s.prefix[s.ngroups];
         if (Cfg<MODE>::kStream) {
             const int nt = s.tprefix[s.ngroups];
             const int D = dp_tiles_per_cta(nt, nct);
             dp_next = c * D;
             dp_end = dp_next + D;
-            const int first_split_tile = nct * D;
-            if (first_split_tile < nt) {
-                const int g = find_group_tile(s, first_split_tile);
-                sk_begin = s.prefix[g] + (first_split_tile - s.tprefix[g]) * group_ktiles<MODE>(p, g);
-            } else {
-                sk_begin = total;
-            }
-            sk_total = total - sk_begin;
             pos = sk_range_begin(c);
             re = sk_range_begin(c + 1);
             state = 0;
@@ -325,11 +384,19 @@ struct WorkIter {
             t = c;
         }
     }
-    // first k-step of CTA cc's split range, and the CTA whose range holds `abs`
-    __device__ int sk_range_begin(int cc) const {
-        return sk_begin + static_cast<int>(static_cast<long>(cc) * sk_total / nct);
+    // first k-step of CTA cc's split range
+    __device__ int sk_range_begin(int cc) const { return sp->rb[cc < 0 ? 0 : (cc > nct ? nct : cc)]; }
+    // The CTA whose split range holds k-step `abs` (abs in the split region):
+    // the largest cc with sk_range_begin(cc) <= abs.
+    __device__ int sk_cta_of(int abs) const {
+        const int* rb = sp->rb;
+        int lo = 0, hi = nct - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (rb[mid] <= abs) lo = mid; else hi = mid - 1;
+        }
+        return lo;
     }
-    __device__ int sk_cta_of(int abs) const { return cta_of(abs - sk_begin, sk_total, nct); }
 
     __device__ bool next(const Params& p, const Sched& s, Work& w) {
         if (Cfg<MODE>::kStream) {
@@ -395,7 +462,14 @@ __device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, uint64_t
     return *static_cast<volatile int*>(&go) != 0;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+// silu(g) * u with CUDA's fast exponential and division intrinsics: their
+// relative error (a few units in the last fp32 place) is far below the bf16
+// rounding that h receives, and the epilogue of a 128-token tile evaluates it
+// 128 times per thread, where the IEEE forms made the CTAs that hold the
+// shared experts' tiles finish several microseconds after the others.
+// Limits: g -> -inf gives -0 (the exponential overflows to +inf, whose
+// reciprocal is 0); g -> +inf gives g.
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 // Order-preserving 16-bit key of the bf16 rounding of v: a larger value has a
 // larger key, and -0 is taken as +0 (they compare equal).  NaN is not ordered.
@@ -586,10 +660,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         abort_sh = 0;
         fence_mbar_init();
     }
-    // The schedule needs only the routing offsets.  They were written two
-    // kernels back on this stream (the permutation, before the gather kernel
-    // or GEMM1 that precedes this launch); that predecessor already waited
-    // for them, so they are complete even while it is still running.
+    // The schedule needs only the routing offsets.  They were written two or
+    // more kernels back on this stream (the permutation, before the gather
+    // kernel or GEMM1's finish that precedes this launch), which every kernel
+    // in between waited for, so they are complete.
     build_schedule<MODE>(p, sched);
     if (threadIdx.x == 0) tstamp(p, MODE, TS_SCHEDULE);
 
@@ -597,8 +671,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int kt_h = p.H / BK, kt_i = p.I / BK;
     int q_issued = 0;                       // k-steps whose loads were issued
     int npre = 0;                           // k-steps whose weight half was prefetched
+    // streaming: every weight byte is read once per launch, so its lines go
+    // first when L2 needs room
+    const bool hint = kStream && p.weights_evict_first;
+    const uint64_t wpol = hint ? l2_policy_evict_first() : 0;
     auto weight_loads = [&](const Work& w, int kt, uint32_t a, uint32_t b, uint32_t full) {
-        auto ld = [&](uint32_t dst, const CUtensorMap* m, int y, int z) { tma_load_3d(dst, m, full, 0, y, z); };
+        auto ld = [&](uint32_t dst, const CUtensorMap* m, int y, int z) {
+            if (hint) tma_load_3d_hint(dst, m, full, 0, y, z, wpol);
+            else tma_load_3d(dst, m, full, 0, y, z);
+        };
         const bool shared = p.offsets != nullptr && w.g == p.E;
         const int kx = kt * BK;
         if (MODE == G1_STREAM || MODE == G1_TILED) {
@@ -1245,45 +1326,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // that GEMM's epilogue: SwiGLU -> h for GEMM1, y for GEMM2, logits for the
 // vocab head.  Running after the GEMM, it reads the partials from a quiet
 // memory system instead of competing with the GEMM's weight stream.
-// One CTA per (split tile, 16-column chunk); 128 threads = the tile's rows.
+// Work items are the (split tile, 16-column chunk) pairs whose chunk holds
+// tokens (token-major argmax: all 8 chunks of 16 vocabulary rows), in tile
+// order; CTA b takes items b, b + grid, ...  128 threads = the tile's rows.
 // timeline row of the finish kernel that follows GEMM mode MODE
 template <int MODE>
 __device__ __forceinline__ void fin_stamp(const Params& p, int slot) {
-    if (blockIdx.y == 0 && threadIdx.x == 0) tstamp(p, 5 + MODE, slot);
+    if (threadIdx.x == 0) tstamp(p, 5 + MODE, slot);
 }
 
 constexpr int FIN_THREADS = BM;
 
+// Grid of the finish kernel: enough CTAs for every item of a typical batch in
+// one round (at most 2*nct - 1 split tiles, each with NMAX/16 chunks), but
+// no more than a few per SM, so that the CTAs start quickly and leave room
+// for the next GEMM's CTAs.
 template <int MODE, int NMAX>
-__global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p) {
-    __shared__ Sched sched;
-    fin_stamp<MODE>(p, TS_ENTRY);
-    // The offsets come from a kernel at least two launches back, which every
-    // kernel of this library waits for before it lets its successor start:
-    // they may be read before this launch's own wait.
-    build_schedule_n<MODE, FIN_THREADS>(p, sched);
-    grid_dep_wait();
-    grid_dep_launch();
-    fin_stamp<MODE>(p, TS_SCHEDULE);
-    WorkIter<MODE> it;
-    it.init(p, sched, 0, p.nct);
-    const int nt = sched.tprefix[sched.ngroups];
-    const int first_split = p.nct * dp_tiles_per_cta(nt, p.nct);
-    const int t = first_split + static_cast<int>(blockIdx.x);
-    if (t >= nt) return;
-    const int g = find_group_tile(sched, t);
+static int finish_grid(int nct) {
+    const int most = 2 * nct * (NMAX / 16);
+    const int cap = (MODE == LM_STREAM ? 16 : 4) * nct;
+    return most < cap ? most : cap;
+}
+
+// One item of the finish kernel: split tile t (n-th tile of group g), chunk ch.
+template <int MODE, int NMAX>
+__device__ __forceinline__ void finish_item(const Params& p, const Sched& sched, const WorkIter<MODE>& it, int g,
+                                            int t, int ch) {
+    constexpr bool kG1 = Cfg<MODE>::kG1;
+    const int slot_floats = BM * NMAX * (kG1 ? 2 : 1);
+    const int r = threadIdx.x;
     const int kt = group_ktiles<MODE>(p, g);
     const int n = t - sched.tprefix[g];
     const int tile_start = sched.prefix[g] + n * kt;
     const int c_first = it.sk_cta_of(tile_start), c_last = it.sk_cta_of(tile_start + kt - 1);
     if (c_first == c_last) return;   // one CTA did the whole tile and stored it
     const int rows = sched.rows[g], row0 = sched.row0[g];
-    const int ch = blockIdx.y;
-    // (token-major argmax: ch = 16 vocabulary rows, all of them)
-    if (!(MODE == LM_STREAM && p.amax_key && NMAX == BM) && ch * 16 >= rows) return;
-    constexpr bool kG1 = Cfg<MODE>::kG1;
-    const int slot_floats = BM * NMAX * (kG1 ? 2 : 1);
-    const int r = threadIdx.x;
     auto slot_of = [&](int c2) -> const float* {
         const int b2 = it.sk_range_begin(c2);
         if (it.sk_range_begin(c2 + 1) <= b2) return nullptr;   // empty range: not a contributor
@@ -1301,7 +1378,6 @@ __global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p)
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             if (ch * 16 + j < rows) argmax_warp_store(p.amax_key, p.V / 16, ch * 16 + j, va[j], r, n, r >> 5, r & 31);
-        fin_stamp<MODE>(p, TS_EXIT);
         return;
     }
     if (MODE == LM_STREAM && p.amax_key) {
@@ -1310,7 +1386,6 @@ __global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p)
             slot_sum<NMAX, 4, false>(slot_of, c_first, c_last, ch, r, va, vb);
             argmax_chunk_store(p.amax_key, p.V / 16, r, va, n * (BM / 16) + ch);
         }
-        fin_stamp<MODE>(p, TS_EXIT);
         return;
     }
     const int rc = rows - ch * 16;   // tokens of this chunk (only those are read)
@@ -1345,6 +1420,64 @@ __global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p)
             }
         } else {
             p.logits[static_cast<size_t>(tok) * p.V + f] = __float2bfloat16_rn(va[j]);
+        }
+    }
+}
+
+template <int MODE, int NMAX>
+__global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p) {
+    __shared__ Sched sched;
+    __shared__ int iprefix[MAX_GROUPS + 1];   // items before group g
+    fin_stamp<MODE>(p, TS_ENTRY);
+    // The offsets come from a kernel at least two launches back, which every
+    // kernel of this library waits for before it lets its successor start:
+    // they may be read before this launch's own wait.
+    build_schedule_n<MODE, FIN_THREADS>(p, sched);
+    const bool tokM = MODE == LM_STREAM && p.amax_key != nullptr && NMAX == BM;
+    const int ng = sched.ngroups;
+    const int nt = sched.tprefix[ng];
+    const int first_split = p.nct * dp_tiles_per_cta(nt, p.nct);
+    auto nchunks = [&](int g) { return tokM ? BM / 16 : (sched.rows[g] + 15) / 16; };
+    // with at most 16 tokens every split tile is one item: item i is split tile i
+    constexpr bool kOneChunk = NMAX == 16;
+    if (!kOneChunk) {
+        for (int g = threadIdx.x; g < ng; g += FIN_THREADS) {
+            const int lo = max(first_split, sched.tprefix[g]), hi = sched.tprefix[g + 1];
+            iprefix[g + 1] = hi > lo ? (hi - lo) * nchunks(g) : 0;
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) warp_scan_groups(iprefix, ng, threadIdx.x);
+        __syncthreads();
+    }
+    const int nitems = kOneChunk ? nt - first_split : iprefix[ng];
+    grid_dep_wait();
+    grid_dep_launch();
+    fin_stamp<MODE>(p, TS_SCHEDULE);
+    WorkIter<MODE> it;
+    it.init(p, sched, 0, p.nct);
+    if constexpr (kOneChunk) {
+        // the grid (2 nct CTAs) covers every split tile: one item per CTA, no
+        // loop (a loop around the item doubles the kernel's register use)
+        const int item = static_cast<int>(blockIdx.x);
+        if (item < nitems) {
+            const int t = first_split + item;
+            finish_item<MODE, NMAX>(p, sched, it, find_group_tile(sched, t), t, 0);
+        }
+    } else {
+#pragma unroll 1
+        for (int item = static_cast<int>(blockIdx.x); item < nitems; item += static_cast<int>(gridDim.x)) {
+            // group of the item: largest g with iprefix[g] <= item (groups
+            // without items have iprefix[g] == iprefix[g + 1] and are never chosen)
+            int lo = 0, hi = ng - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (iprefix[mid] <= item) lo = mid; else hi = mid - 1;
+            }
+            const int g = lo;
+            const int nch = nchunks(g);
+            const int local = item - iprefix[g];
+            finish_item<MODE, NMAX>(p, sched, it, g, max(first_split, sched.tprefix[g]) + local / nch,
+                                    local - (local / nch) * nch);
         }
     }
     fin_stamp<MODE>(p, TS_EXIT);
@@ -1390,6 +1523,16 @@ __global__ void __launch_bounds__(256) ffn_prep_kernel(const __nv_bfloat16* __re
 }
 
 // ------------------------------------------------------------ host side
+// MOESPEC_NO_EVICT_FIRST=1 loads the streamed weights with the default L2
+// policy (for comparison).
+static int evict_first_allowed() {
+    static const int on = [] {
+        const char* e = getenv("MOESPEC_NO_EVICT_FIRST");
+        return (e && e[0] == '1') ? 0 : 1;
+    }();
+    return on;
+}
+
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -1488,11 +1631,13 @@ static ms_status launch_gemm_pair(int id, const Maps& maps, Params prm, cudaStre
 template <int MODE, int NMAX>
 static ms_status launch_stream_n(int id, const Maps& maps, Params prm, cudaStream_t s) {
     prm.nct = num_sms();
+    if (prm.nct > MAX_CTAS) return MS_ERR_UNSUPPORTED;   // the schedule keeps one range per CTA
+    prm.weights_evict_first = evict_first_allowed();
     ms_status st = launch_gemm<MODE, NMAX>(id, maps, prm, s);
     if (st != MS_OK) return st;
     // fewer than 2 nct tiles are split; one CTA per (tile, 16-column chunk)
-    return launch(K_FFN_FINISH, ffn_finish_kernel<MODE, NMAX>, dim3(2 * num_sms(), NMAX / 16), dim3(FIN_THREADS),
-                  0, s, prm);
+    return launch(K_FFN_FINISH, ffn_finish_kernel<MODE, NMAX>, dim3(finish_grid<MODE, NMAX>(prm.nct)),
+                  dim3(FIN_THREADS), 0, s, prm);
 }
 
 // The streaming GEMM followed by the kernel that finishes its split tiles.
