@@ -125,11 +125,11 @@ struct Sched {
     int tprefix[MAX_GROUPS + 1];  // streaming: output tiles before group g
     int rows[MAX_GROUPS];
     int row0[MAX_GROUPS];
-    // streaming: the split region is the k-steps [sk_begin, total); cpre[g] is
-    // the cost (step_cost units) of its k-steps that lie before group g, and
-    // CTA c's split range is the k-steps [rb[c], rb[c + 1])
+    // streaming: fcp[g] is the cost (step_cost units) of all k-steps before
+    // group g; the split region is the k-steps [sk_begin, total), and CTA c's
+    // split range is the k-steps [rb[c], rb[c + 1])
     int sk_begin;
-    int cpre[MAX_GROUPS + 1];
+    int fcp[MAX_GROUPS + 1];
     int rb[MAX_CTAS + 1];
 };
 
@@ -247,38 +247,36 @@ __device__ void build_schedule_n(const Params& p, Sched& s) {
         }
         s.prefix[g + 1] = units;   // scanned below
         s.tprefix[g + 1] = tiles;
+        if (Cfg<MODE>::kStream) s.fcp[g + 1] = units * step_cost<MODE>(s, g);
     }
     __syncthreads();
     if (tid < 32) warp_scan_groups(s.prefix, ng, tid);
     else if (tid < 64) warp_scan_groups(s.tprefix, ng, tid - 32);
+    else if (Cfg<MODE>::kStream && tid < 96) warp_scan_groups(s.fcp, ng, tid - 64);
     __syncthreads();
     if (Cfg<MODE>::kStream) {
         // the split region: the tiles after the nct * D whole tiles
+        __shared__ int skb_cost;   // cost of the k-steps before the split region
         if (tid == 0) {
             const int nt = s.tprefix[ng];
             const int fs = p.nct * dp_tiles_per_cta(nt, p.nct);
-            int skb = s.prefix[ng];
+            int skb = s.prefix[ng], cskb = s.fcp[ng];
             if (fs < nt) {
                 const int g = find_group_tile(s, fs);
                 skb = s.prefix[g] + (fs - s.tprefix[g]) * group_ktiles<MODE>(p, g);
+                cskb = s.fcp[g] + (skb - s.prefix[g]) * step_cost<MODE>(s, g);
             }
             s.sk_begin = skb;
+            skb_cost = cskb;
         }
         __syncthreads();
-        for (int g = tid; g < ng; g += NT) {
-            const int lo = max(s.prefix[g], s.sk_begin), hi = s.prefix[g + 1];
-            s.cpre[g + 1] = hi > lo ? (hi - lo) * step_cost<MODE>(s, g) : 0;
-        }
-        __syncthreads();
-        if (tid < 32) warp_scan_groups(s.cpre, ng, tid);
-        __syncthreads();
-        // CTA c's range starts at the first k-step whose cost prefix reaches
-        // c/nct of the region's cost
+        // CTA c's range starts at the first k-step whose cost from the start
+        // of the split region reaches c/nct of the region's cost
         const int nct = p.nct, total = s.prefix[ng];
-        const long long C = s.cpre[ng];
+        const long long C0 = skb_cost, C = s.fcp[ng] - C0;
         // 32-bit arithmetic when the scaled costs fit (every layer of this
         // model); 64-bit division is several times slower
-        const bool narrow = C * nct < (1LL << 31);
+        const bool narrow = static_cast<long long>(s.fcp[ng]) * nct < (1LL << 31);
         for (int c = tid; c <= nct; c += NT) {
             int b;
             if (c == 0 || C == 0) {
@@ -286,18 +284,18 @@ __device__ void build_schedule_n(const Params& p, Sched& s) {
             } else if (c == nct) {
                 b = total;
             } else {
-                const long long x = C * c;   // the target cost, times nct
-                int lo = 0, hi = ng - 1;     // largest g with cpre[g] * nct <= x
+                const long long x = C * c + C0 * nct;   // the target cost, times nct
+                int lo = 0, hi = ng - 1;                // largest g with fcp[g] * nct <= x
                 while (lo < hi) {
                     const int mid = (lo + hi + 1) >> 1;
-                    if (static_cast<long long>(s.cpre[mid]) * nct <= x) lo = mid; else hi = mid - 1;
+                    if (static_cast<long long>(s.fcp[mid]) * nct <= x) lo = mid; else hi = mid - 1;
                 }
-                const long long num = x - static_cast<long long>(s.cpre[lo]) * nct;
+                const long long num = x - static_cast<long long>(s.fcp[lo]) * nct;
                 const long long den = static_cast<long long>(nct) * step_cost<MODE>(s, lo);
                 const int d = narrow ? static_cast<int>((static_cast<uint32_t>(num) + static_cast<uint32_t>(den) - 1u) /
                                                         static_cast<uint32_t>(den))
                                      : static_cast<int>((num + den - 1) / den);
-                b = max(s.prefix[lo], s.sk_begin) + d;
+                b = max(s.prefix[lo] + d, s.sk_begin);
             }
             s.rb[c] = b;
         }
@@ -465,8 +463,7 @@ __device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, uint64_t
 // silu(g) * u with CUDA's fast exponential and division intrinsics: their
 // relative error (a few units in the last fp32 place) is far below the bf16
 // rounding that h receives, and the epilogue of a 128-token tile evaluates it
-// 128 times per thread, where the IEEE forms made the CTAs that hold the
-// shared experts' tiles finish several microseconds after the others.
+// 128 times per thread (the IEEE forms cost about 1 us per such tile).
 // Limits: g -> -inf gives -0 (the exponential overflows to +inf, whose
 // reciprocal is 0); g -> +inf gives g.
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
