@@ -218,17 +218,19 @@ __global__ void __launch_bounds__(256) route_tiled_kernel(const __nv_bfloat16* _
     }
 }
 
-// Small T: one cluster of RC_CTAS CTAs per token.  CTA r computes the logits
-// of experts [r*E/RC_CTAS, (r+1)*E/RC_CTAS) -- one warp per expert, float4
-// loads of W_r spread over RC_CTAS SMs -- and stores them into CTA 0's shared
-// memory (distributed shared memory); after the cluster barrier CTA 0 runs the
-// softmax and top-k.  With NORM the CTAs first RMS-normalise the fp32 residual
-// row themselves (eps, unit gain) and CTA 0 writes the bf16 result, so the
-// layer needs no separate normalisation kernel.
+// Small T: one cluster of RC_CTAS CTAs per TPC tokens.  CTA r computes the
+// logits of experts [r*E/RC_CTAS, (r+1)*E/RC_CTAS) for the cluster's tokens --
+// one warp per expert, whose W_r row is read once (float4 loads) and used for
+// every token -- and stores them into CTA 0's shared memory (distributed
+// shared memory); after the cluster barrier CTA 0 runs the softmax and top-k,
+// one warp per token.  With NORM the CTAs first RMS-normalise the fp32
+// residual rows themselves (eps, unit gain) and CTA 0 writes the bf16 result,
+// so the layer needs no separate normalisation kernel.  Each token's logits
+// are summed in the same order whatever TPC is.
 constexpr int RC_CTAS = 8;
 constexpr int RC_WPRE = 12;   // float4 of a router row per lane kept in registers (H <= 1536)
 
-template <bool NORM>
+template <bool NORM, int TPC>
 __global__ void __launch_bounds__(256) route_cluster_kernel(const void* __restrict__ xin,
                                                             const float* __restrict__ wr,
                                                             const float* __restrict__ bias, int T, int H,
@@ -236,19 +238,19 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(const void* __restri
                                                             int32_t* __restrict__ idx, float* __restrict__ w,
                                                             __nv_bfloat16* __restrict__ xhat_out) {
     extern __shared__ float smem[];
-    float* xs = smem;        // [H] the token's normalised activation (bf16 values)
-    float* z = smem + H;     // [E] logits, filled by every CTA of the cluster
-    __shared__ float red[8];
-    grid_dep_wait();
-    grid_dep_launch();
+    float* xs = smem;            // [TPC][H] the tokens' normalised activations (bf16 values)
+    float* z = smem + TPC * H;   // [TPC][E] logits, filled by every CTA of the cluster
+    __shared__ float red[TPC][8];
     const uint32_t rank = cluster_rank();
-    const int t = blockIdx.y;
+    const int t0 = static_cast<int>(blockIdx.y) * TPC;
+    const int nt = T - t0 < TPC ? T - t0 : TPC;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int per = (E + RC_CTAS - 1) / RC_CTAS;
     const int e0 = static_cast<int>(rank) * per;
     const int e1 = e0 + per < E ? e0 + per : E;
-    // this warp's first router row, loaded together with the activation row
-    // (independent loads, one round trip) when it fits the registers
+    // this warp's first router row, loaded before the dependency wait when it
+    // fits the registers: no kernel of this library writes the router weights,
+    // and a kernel of any other origin has completed before this one starts
     const bool wpre = H / 4 <= 32 * RC_WPRE && e0 + warp < e1;
     float4 wv[RC_WPRE];
     if (wpre) {
@@ -259,97 +261,152 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(const void* __restri
             wv[j] = h4 < H / 4 ? __ldg(wrow + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
+    grid_dep_wait();
+    grid_dep_launch();
     if (NORM) {
-        const float4* row = reinterpret_cast<const float4*>(static_cast<const float*>(xin) + static_cast<size_t>(t) * H);
-        float ss = 0.f;
-        for (int i = threadIdx.x; i < H / 4; i += blockDim.x) {
-            const float4 v = __ldg(row + i);
-            ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-        }
-        ss = warp_sum(ss);
-        if (lane == 0) red[warp] = ss;
-        __syncthreads();
-        float tot = 0.f;
+        const float* xf = static_cast<const float*>(xin);
+        float ss[TPC];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) tot += red[i];
-        const float inv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+        for (int tt = 0; tt < TPC; ++tt) ss[tt] = 0.f;
         for (int i = threadIdx.x; i < H / 4; i += blockDim.x) {
-            const float4 v = __ldg(row + i);
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x * inv, v.y * inv);
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z * inv, v.w * inv);
-            xs[4 * i] = __low2float(lo);
-            xs[4 * i + 1] = __high2float(lo);
-            xs[4 * i + 2] = __low2float(hi);
-            xs[4 * i + 3] = __high2float(hi);
-            if (rank == 0) {
-                __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(xhat_out + static_cast<size_t>(t) * H);
-                o[2 * i] = lo;
-                o[2 * i + 1] = hi;
+#pragma unroll
+            for (int tt = 0; tt < TPC; ++tt) {
+                if (tt >= nt) break;
+                const float4 v = __ldg(reinterpret_cast<const float4*>(xf + static_cast<size_t>(t0 + tt) * H) + i);
+                ss[tt] += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+            }
+        }
+#pragma unroll
+        for (int tt = 0; tt < TPC; ++tt) {
+            ss[tt] = warp_sum(ss[tt]);
+            if (lane == 0) red[tt][warp] = ss[tt];
+        }
+        __syncthreads();
+        float inv[TPC];
+#pragma unroll
+        for (int tt = 0; tt < TPC; ++tt) {
+            float tot = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) tot += red[tt][i];
+            inv[tt] = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+        }
+        for (int i = threadIdx.x; i < H / 4; i += blockDim.x) {
+#pragma unroll
+            for (int tt = 0; tt < TPC; ++tt) {
+                if (tt >= nt) break;
+                const float4 v = __ldg(reinterpret_cast<const float4*>(xf + static_cast<size_t>(t0 + tt) * H) + i);
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x * inv[tt], v.y * inv[tt]);
+                const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z * inv[tt], v.w * inv[tt]);
+                float* x4 = xs + tt * H + 4 * i;
+                x4[0] = __low2float(lo);
+                x4[1] = __high2float(lo);
+                x4[2] = __low2float(hi);
+                x4[3] = __high2float(hi);
+                if (rank == 0) {
+                    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(xhat_out + static_cast<size_t>(t0 + tt) * H);
+                    o[2 * i] = lo;
+                    o[2 * i + 1] = hi;
+                }
             }
         }
     } else {
-        const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(xin) + static_cast<size_t>(t) * H);
         for (int i = threadIdx.x; i < H / 8; i += blockDim.x) {
-            const uint4 u = __ldg(xr + i);
-            const uint32_t q[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                xs[8 * i + 2 * j] = __uint_as_float(q[j] << 16);
-                xs[8 * i + 2 * j + 1] = __uint_as_float(q[j] & 0xffff0000u);
+            for (int tt = 0; tt < TPC; ++tt) {
+                if (tt >= nt) break;
+                const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(xin) +
+                                                                     static_cast<size_t>(t0 + tt) * H) + i);
+                const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    xs[tt * H + 8 * i + 2 * j] = __uint_as_float(q[j] << 16);
+                    xs[tt * H + 8 * i + 2 * j + 1] = __uint_as_float(q[j] & 0xffff0000u);
+                }
             }
         }
     }
     __syncthreads();
     for (int e = e0 + warp; e < e1; e += 8) {
         const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * H);
-        float acc = 0.f;
+        float acc[TPC];
+#pragma unroll
+        for (int tt = 0; tt < TPC; ++tt) acc[tt] = 0.f;
         if (wpre && e == e0 + warp) {
 #pragma unroll
             for (int j = 0; j < RC_WPRE; ++j) {
                 const int h4 = lane + 32 * j;
                 if (h4 < H / 4) {
-                    const float4 b = *reinterpret_cast<const float4*>(xs + 4 * h4);
-                    acc = fmaf(wv[j].x, b.x, acc);
-                    acc = fmaf(wv[j].y, b.y, acc);
-                    acc = fmaf(wv[j].z, b.z, acc);
-                    acc = fmaf(wv[j].w, b.w, acc);
+#pragma unroll
+                    for (int tt = 0; tt < TPC; ++tt) {
+                        const float4 b = *reinterpret_cast<const float4*>(xs + tt * H + 4 * h4);
+                        acc[tt] = fmaf(wv[j].x, b.x, acc[tt]);
+                        acc[tt] = fmaf(wv[j].y, b.y, acc[tt]);
+                        acc[tt] = fmaf(wv[j].z, b.z, acc[tt]);
+                        acc[tt] = fmaf(wv[j].w, b.w, acc[tt]);
+                    }
                 }
             }
         } else {
 #pragma unroll 4
             for (int h4 = lane; h4 < H / 4; h4 += 32) {
                 const float4 a = __ldg(wrow + h4);
-                const float4 b = *reinterpret_cast<const float4*>(xs + 4 * h4);
-                acc = fmaf(a.x, b.x, acc);
-                acc = fmaf(a.y, b.y, acc);
-                acc = fmaf(a.z, b.z, acc);
-                acc = fmaf(a.w, b.w, acc);
+#pragma unroll
+                for (int tt = 0; tt < TPC; ++tt) {
+                    const float4 b = *reinterpret_cast<const float4*>(xs + tt * H + 4 * h4);
+                    acc[tt] = fmaf(a.x, b.x, acc[tt]);
+                    acc[tt] = fmaf(a.y, b.y, acc[tt]);
+                    acc[tt] = fmaf(a.z, b.z, acc[tt]);
+                    acc[tt] = fmaf(a.w, b.w, acc[tt]);
+                }
             }
         }
-        acc = warp_sum(acc);
-        if (lane == 0) st_cluster_f32(&z[e], 0, bias ? acc + __ldg(bias + static_cast<size_t>(t) * E + e) : acc);
+#pragma unroll
+        for (int tt = 0; tt < TPC; ++tt) {
+            const float sum = warp_sum(acc[tt]);
+            if (lane == 0 && tt < nt)
+                st_cluster_f32(&z[tt * E + e], 0,
+                               bias ? sum + __ldg(bias + static_cast<size_t>(t0 + tt) * E + e) : sum);
+        }
     }
     cluster_sync_all();
-    if (rank == 0 && warp == 0)
-        warp_topk_softmax(z, E, k, renorm, idx + static_cast<size_t>(t) * k, w + static_cast<size_t>(t) * k, lane);
+    if (rank == 0 && warp < nt)
+        warp_topk_softmax(z + warp * E, E, k, renorm, idx + static_cast<size_t>(t0 + warp) * k,
+                          w + static_cast<size_t>(t0 + warp) * k, lane);
+}
+
+// Tokens per cluster: one for small batches (the latency of one token's
+// chain), four above 32 tokens, where a W_r row read once serves four tokens
+// and the grid has a quarter of the CTAs.
+constexpr int RC_TPC = 4;
+
+template <bool NORM>
+static ms_status route_cluster_launch_t(const void* xin, float eps, const float* wr, const float* bias, int T, int H,
+                                        int E, int k, int renorm, int32_t* idx, float* w, __nv_bfloat16* xo,
+                                        cudaStream_t s) {
+    static bool set = false;
+    if (!set) {
+        cudaFuncSetAttribute(route_cluster_kernel<NORM, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaFuncSetAttribute(route_cluster_kernel<NORM, RC_TPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             200 * 1024);
+        set = true;
+    }
+    if (T > 32) {
+        const size_t smem = sizeof(float) * static_cast<size_t>(RC_TPC) * (H + E);
+        return launch_cluster(K_ROUTE_CLUSTER, route_cluster_kernel<NORM, RC_TPC>,
+                              dim3(RC_CTAS, (T + RC_TPC - 1) / RC_TPC), dim3(256), smem, s, RC_CTAS, xin, wr, bias,
+                              T, H, E, k, renorm, eps, idx, w, xo);
+    }
+    const size_t smem = sizeof(float) * static_cast<size_t>(H + E);
+    return launch_cluster(K_ROUTE_CLUSTER, route_cluster_kernel<NORM, 1>, dim3(RC_CTAS, T), dim3(256), smem, s,
+                          RC_CTAS, xin, wr, bias, T, H, E, k, renorm, eps, idx, w, xo);
 }
 
 ms_status route_cluster_launch(const void* xin, bool norm, float eps, const float* wr, const float* bias, int T,
                                int H, int E, int k, int renorm, int32_t* idx, float* w, void* xhat_out,
                                cudaStream_t s) {
-    const size_t smem = sizeof(float) * static_cast<size_t>(H + E);
-    static bool set = false;
-    if (!set) {
-        cudaFuncSetAttribute(route_cluster_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        cudaFuncSetAttribute(route_cluster_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        set = true;
-    }
     auto* xo = reinterpret_cast<__nv_bfloat16*>(xhat_out);
-    if (norm)
-        return launch_cluster(K_ROUTE_CLUSTER, route_cluster_kernel<true>, dim3(RC_CTAS, T), dim3(256), smem, s,
-                              RC_CTAS, xin, wr, bias, T, H, E, k, renorm, eps, idx, w, xo);
-    return launch_cluster(K_ROUTE_CLUSTER, route_cluster_kernel<false>, dim3(RC_CTAS, T), dim3(256), smem, s,
-                          RC_CTAS, xin, wr, bias, T, H, E, k, renorm, eps, idx, w, xo);
+    if (norm) return route_cluster_launch_t<true>(xin, eps, wr, bias, T, H, E, k, renorm, idx, w, xo, s);
+    return route_cluster_launch_t<false>(xin, eps, wr, bias, T, H, E, k, renorm, idx, w, xo, s);
 }
 
 ms_status route_launch(const void* x, const float* wr, const float* bias, int T, int H, int E,

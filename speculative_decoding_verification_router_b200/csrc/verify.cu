@@ -204,10 +204,30 @@ ms_status verify_keys_launch(const unsigned long long* keys, int ld, int B, int 
 constexpr int VC_THREADS = 512;
 constexpr int VC_MAX = 16;
 
+// Merge the elements of one 16-byte vector (index i0 for its first element),
+// converting each as it is compared, so that a thread keeps only the raw
+// vectors of its loads in flight in registers.
+__device__ __forceinline__ void merge_vec(float& bv, int& bi, const uint4& r, int i0, const __nv_bfloat16*) {
+    const uint32_t q[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        argmax_merge(bv, bi, __uint_as_float(q[j] << 16), i0 + 2 * j);
+        argmax_merge(bv, bi, __uint_as_float(q[j] & 0xffff0000u), i0 + 2 * j + 1);
+    }
+}
+__device__ __forceinline__ void merge_vec(float& bv, int& bi, const uint4& r, int i0, const float*) {
+    argmax_merge(bv, bi, __uint_as_float(r.x), i0);
+    argmax_merge(bv, bi, __uint_as_float(r.y), i0 + 1);
+    argmax_merge(bv, bi, __uint_as_float(r.z), i0 + 2);
+    argmax_merge(bv, bi, __uint_as_float(r.w), i0 + 3);
+}
+
 // UNROLL: 16-byte loads in flight per thread -- 8 for small batches (latency:
-// one round trip for a 64 KB chunk), 4 for large ones (occupancy).
+// one round trip for a 64 KB chunk), 4 for large ones, where four 512-thread
+// CTAs per SM must fit for the whole grid to be resident at once (B = 32,
+// K = 3: 512 CTAs), which holds the kernel to 32 registers.
 template <typename TL, int UNROLL>
-__global__ void __launch_bounds__(VC_THREADS) verify_cluster_kernel(const TL* __restrict__ logits, int K, int V,
+__global__ void __launch_bounds__(VC_THREADS, UNROLL == 4 ? 4 : 1) verify_cluster_kernel(const TL* __restrict__ logits, int K, int V,
                                                                     int P, int chunk, int vec_ok,
                                                                     const int32_t* __restrict__ draft,
                                                                     int32_t* __restrict__ argmax,
@@ -233,20 +253,19 @@ __global__ void __launch_bounds__(VC_THREADS) verify_cluster_kernel(const TL* __
         int tail_begin = begin;
         if (vec_ok && end > begin) {
             const int nvec = (end - begin) / VEC;
+            // begin is a multiple of VEC and the row starts 16-byte aligned
+            const uint4* rv = reinterpret_cast<const uint4*>(row + begin);
             for (int q0 = threadIdx.x; q0 < nvec; q0 += UNROLL * VC_THREADS) {
-                float v[UNROLL][VEC];
+                uint4 raw[UNROLL];
 #pragma unroll
                 for (int u = 0; u < UNROLL; ++u) {
                     const int q = q0 + u * VC_THREADS;
-                    if (q < nvec) vec_load(row + begin + q * VEC, v[u]);
+                    if (q < nvec) raw[u] = __ldg(rv + q);
                 }
 #pragma unroll
                 for (int u = 0; u < UNROLL; ++u) {
                     const int q = q0 + u * VC_THREADS;
-                    if (q < nvec) {
-#pragma unroll
-                        for (int e = 0; e < VEC; ++e) argmax_merge(bv, bi, v[u][e], begin + q * VEC + e);
-                    }
+                    if (q < nvec) merge_vec(bv, bi, raw[u], begin + q * VEC, row);
                 }
             }
             tail_begin = begin + nvec * VEC;
