@@ -11,12 +11,13 @@
 //  * streaming (verify-sized T <= 128): the weights are the M = 128 operand
 //    and the tokens of one expert the N operand (N = rows rounded up to 16).
 //    Every CTA takes the same number of whole output tiles, all but the last
-//    round; the k-steps of the remaining tiles are divided into equal
-//    contiguous ranges, one per CTA, so every SM streams the same number of
-//    weight bytes ("stream-K").  A CTA's part of a split tile goes to an fp32
-//    partial slot; ffn_finish_kernel, launched after the GEMM, sums the two
-//    or three parts of each split tile in CTA order (deterministic, no CTA
-//    ever waits on another) and applies the epilogue.
+//    round; the k-steps of the remaining tiles are divided into contiguous
+//    ranges, one per CTA, of equal cost (weight bytes plus token-box bytes),
+//    so every SM moves the same amount of data ("stream-K").  Weight tiles
+//    are loaded with an L2 evict-first policy.  A CTA's part of a split tile
+//    goes to an fp32 partial slot; ffn_finish_kernel, launched after the
+//    GEMM, sums the two to four parts of each split tile in CTA order
+//    (deterministic, no CTA ever waits on another) and applies the epilogue.
 //    For GEMM1 the gate and up rows of the same 128 features accumulate into
 //    two TMEM buffers in the same lanes, so SwiGLU is done in registers.
 //  * tiled (prefill-sized T): the tokens of one expert are the M = 128
