@@ -81,6 +81,35 @@ def test_expert_ffn_flags_oversized_group(ms):
     assert_close(host(ysh), rs, what="y_shared beside a rejected group")
 
 
+@pytest.mark.parametrize("pattern", ["head_heavy", "one_full_expert"])
+def test_expert_ffn_unequal_group_sizes(ms, pattern):
+    # 128 tokens whose experts receive very different token counts.  The
+    # streaming schedule cuts its split ranges at equal data cost (weights
+    # plus 16-row token boxes), so a range over a 128-token group holds fewer
+    # k-steps than one over a 2-token group; the results must not depend on it.
+    shp = synth.VERIFY_B32
+    T, k, E = shp.T, shp.k, shp.E
+    lw = synth.layer_weights(shp, 3)
+    rng = synth.stream(3, f"unequal_groups_{pattern}")
+    if pattern == "head_heavy":
+        p = (E - np.arange(E, dtype=np.float64)) ** 4
+        idx = np.stack([rng.choice(E, k, replace=False, p=p / p.sum()) for _ in range(T)])
+    else:
+        # expert 0 in every token's set, the other five drawn uniformly
+        idx = np.stack([np.concatenate([[0], 1 + rng.choice(E - 1, k - 1, replace=False)]) for _ in range(T)])
+    idx = idx.astype(np.int32)
+    off, perm, _ = oracle.permute(idx, E)
+    counts = np.diff(off)
+    assert counts.max() >= 48 and counts[counts > 0].min() <= 4   # the spread the case is about
+    xb = synth.normal_bf16(3, f"unequal_groups_x_{pattern}", (T, shp.H), 1.0)
+    wgu, wd, wsgu, wsd = _weights_dev(lw)
+    y, ysh = ms.expert_ffn(dev(xb), dev(off), dev(perm), wgu, wd, wsgu, wsd, k)
+    torch.cuda.synchronize()
+    xw = oracle.widen_bf16(xb)
+    assert_close(host(y), oracle.expert_ffn_routed(xw, lw.w_gate_up, lw.w_down, off, perm, k), what="y_perm")
+    assert_close(host(ysh), oracle.expert_ffn_shared(xw, lw.ws_gate_up, lw.ws_down), what="y_shared")
+
+
 @pytest.mark.parametrize("T", [129, 300])
 def test_expert_ffn_tiled_ragged(ms, T):
     # the tiled (large-T) schedule on small shapes, with a ragged last tile
