@@ -227,12 +227,10 @@ __device__ __forceinline__ void merge_vec(float& bv, int& bi, const uint4& r, in
 // CTAs per SM must fit for the whole grid to be resident at once (B = 32,
 // K = 3: 512 CTAs), which holds the kernel to 32 registers.
 template <typename TL, int UNROLL>
-__global__ void __launch_bounds__(VC_THREADS, UNROLL == 4 ? 4 : 1) verify_cluster_kernel(const TL* __restrict__ logits, int K, int V,
-                                                                    int P, int chunk, int vec_ok,
-                                                                    const int32_t* __restrict__ draft,
-                                                                    int32_t* __restrict__ argmax,
-                                                                    int32_t* __restrict__ committed,
-                                                                    int32_t* __restrict__ n_committed) {
+__global__ void __launch_bounds__(VC_THREADS, UNROLL == 4 ? 4 : 1)
+    verify_cluster_kernel(const TL* __restrict__ logits, int K, int V, int P, int chunk, int vec_ok,
+                          const int32_t* __restrict__ draft, int32_t* __restrict__ argmax,
+                          int32_t* __restrict__ committed, int32_t* __restrict__ n_committed) {
     constexpr int VEC = 16 / sizeof(TL);
     __shared__ float cv[VC_MAX];
     __shared__ int ci[VC_MAX];
