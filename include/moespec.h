@@ -61,7 +61,11 @@ typedef enum {
     MS_ERR_WORKSPACE = -3,     /* ws missing or smaller than the size query   */
     MS_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed            */
     MS_ERR_TIMEOUT = -5,       /* a device-side bounded wait ran out           */
-    MS_ERR_DEVICE_INDEX = -6   /* a kernel saw an index outside its range      */
+    MS_ERR_DEVICE_INDEX = -6,  /* a kernel saw an index outside its range      */
+    MS_ERR_DRAIN_TIMEOUT = -7  /* after a timeout, a kernel's wait for its own
+                                  in-flight copies/MMAs ran out as well; it
+                                  exited without releasing its tensor memory:
+                                  the device state is undefined, reset it    */
 } ms_status;
 
 typedef enum { MS_F32 = 0, MS_BF16 = 1 } ms_dtype;
@@ -111,6 +115,10 @@ MS_API ms_status moe_permute(const int32_t* topk_idx, int T, int k, int E,
 MS_API ms_status moe_pack_weights(const void* w, int n, int rows, int cols, void* packed, void* stream);
 
 /* a3  Expert FFN: every routed row and the shared experts, SwiGLU.
+ * The experts are the decoder's 64 routed and two shared experts (clawpit.io,
+ * "Lean architecture with a compressed encoder"; aikraft.ru, "Архитектура и
+ * эффективность": 64 routed experts); the pages do not describe an expert's
+ * inside, and SwiGLU is the conventional DeepSeek-MoE expert.
  * All four weight arguments are in the packed layout of moe_pack_weights
  * (w_gate_up: n=E, rows=2I, cols=H; w_down: n=E, rows=H, cols=I; shared: n=S).
  * For grouped row r of expert e (token t = perm_token[r]):
@@ -126,6 +134,9 @@ MS_API ms_status moe_pack_weights(const void* w, int n, int rows, int cols, void
  * expert_offsets must describe groups inside [0, T*k) of at most T rows
  * each (a token reaches an expert at most once); a group that does not is
  * skipped and flagged MS_ERR_DEVICE_INDEX in the status word.
+ * Weights in the plain [E,2I,H] / [E,H,I] row-major layout (not passed
+ * through moe_pack_weights) are NOT detected: both layouts hold the same
+ * number of bf16 values, and the call then returns MS_OK with wrong results.
  * Scratch: moe_expert_ffn_workspace_size(...) bytes; the status word of
  * the bounded waits lives at its start (see ms_device_status). */
 MS_API size_t moe_expert_ffn_workspace_size(int T, int H, int E, int I, int S, int k);
@@ -137,6 +148,11 @@ MS_API ms_status moe_expert_ffn(const void* xhat, const int32_t* expert_offsets,
                          void* ws, size_t ws_bytes, void* stream);
 
 /* a4  Combine: gate-weighted un-permute plus residual.
+ * Each token's output is the weighted sum of its top-k routed experts plus
+ * the two shared experts (clawpit.io, "Lean architecture with a compressed
+ * encoder": 64 routed experts, two shared experts, top-6 routing); the
+ * shared experts enter with weight 1 and the residual stream is added, the
+ * conventional DeepSeek-MoE block (the pages give no formula).
  * out[t,:] = sum_{j<k} topk_w[t,j] * y_perm[slot_of[t,j],:] + y_shared[t,:]
  *            + residual[t,:]            (fp32, in that order)
  * y_perm: [T*k,H] fp32 or bf16.  y_shared, residual: [T,H] fp32 or NULL.

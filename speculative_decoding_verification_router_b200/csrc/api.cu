@@ -264,6 +264,7 @@ const char* ms_status_string(ms_status s) {
         case MS_ERR_CUDA: return "CUDA error";
         case MS_ERR_TIMEOUT: return "device-side bounded wait timed out";
         case MS_ERR_DEVICE_INDEX: return "device-side index out of range";
+        case MS_ERR_DRAIN_TIMEOUT: return "device-side drain after a timeout ran out (device state undefined)";
     }
     return "unknown status";
 }

@@ -632,6 +632,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __shared__ __align__(8) uint64_t bar_full[ST], bar_empty[ST], bar_tfull[2], bar_tempty[2], bar_drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
+    __shared__ volatile int drain_fail_sh;   // a drain wait ran out: TMEM may still be in use
     __shared__ int go_sh[2];
     __shared__ Sched sched;
 
@@ -656,6 +657,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         mbar_init(smem_addr(&bar_drain), 1);
         abort_sh = 0;
+        drain_fail_sh = 0;
         fence_mbar_init();
     }
     // The schedule needs only the routing offsets.  They were written two or
@@ -811,7 +813,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int q_last = s2 + ((q_end - 1 - s2) / ST) * ST;
             volatile int never = 0;
             if (!mbar_wait(smem_addr(&bar_full[s2]), static_cast<uint32_t>(q_last / ST) & 1u, lim, &never))
-                report_status(p.status, MS_ERR_TIMEOUT);
+                drain_failed(p.status, drain_fail_sh);
         }
         tstamp(p, MODE, TS_PRODUCER_DONE);
       }
@@ -875,7 +877,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // drain: all MMAs issued by this thread complete before TMEM is freed
         mma_commit(smem_addr(&bar_drain));
         volatile int never = 0;
-        if (!mbar_wait(smem_addr(&bar_drain), 0, lim, &never)) report_status(p.status, MS_ERR_TIMEOUT);
+        if (!mbar_wait(smem_addr(&bar_drain), 0, lim, &never)) drain_failed(p.status, drain_fail_sh);
       }
       __syncwarp();
     } else {
@@ -1034,7 +1036,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+    // After a drain wait that ran out, loads or MMAs of this CTA may still be
+    // in flight: its TMEM is left allocated rather than handed to another CTA
+    // while an MMA may still write it (MS_ERR_DRAIN_TIMEOUT is recorded; the
+    // device is then in an undefined state and the caller must reset it).
+    if (warp == 1 && !drain_fail_sh) tmem_dealloc(tmem_base, TMEM_COLS);
     if (threadIdx.x == 32) tstamp(p, MODE, TS_EXIT);
 }
 
@@ -1066,6 +1072,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __shared__ __align__(8) uint64_t bar_full[ST], bar_empty[ST], bar_tfull[2], bar_tempty[2], bar_drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
+    __shared__ volatile int drain_fail_sh;   // a drain wait ran out: TMEM may still be in use
     __shared__ int go_sh[2];
     __shared__ Sched sched;
 
@@ -1091,6 +1098,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         mbar_init(smem_addr(&bar_drain), 1);
         abort_sh = 0;
+        drain_fail_sh = 0;
         fence_mbar_init();
     }
     build_schedule<MODE>(p, sched);
@@ -1161,7 +1169,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int q_last = s2 + ((q - 1 - s2) / ST) * ST;
             volatile int never = 0;
             if (!mbar_wait(smem_addr(&bar_empty[s2]), static_cast<uint32_t>(q_last / ST) & 1u, lim, &never))
-                report_status(p.status, MS_ERR_TIMEOUT);
+                drain_failed(p.status, drain_fail_sh);
         }
         tstamp(p, MODE, TS_PRODUCER_DONE);
       }
@@ -1217,7 +1225,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // drain: every pair MMA issued by this thread completes before TMEM is freed
             mma_commit_pair(mapa_shared(smem_addr(&bar_drain), 0));
             volatile int never = 0;
-            if (!mbar_wait(smem_addr(&bar_drain), 0, lim, &never)) report_status(p.status, MS_ERR_TIMEOUT);
+            if (!mbar_wait(smem_addr(&bar_drain), 0, lim, &never)) drain_failed(p.status, drain_fail_sh);
         }
       }
       __syncwarp();
@@ -1314,7 +1322,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // CTA frees either before both got here
     cluster_sync_all();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    // the pair's TMEM is released by both CTAs together, and only if neither
+    // CTA's drain wait ran out (see ffn_gemm_kernel)
+    if (warp == 1 && !drain_fail_sh && !peer_flag(&drain_fail_sh)) tmem_dealloc_pair(tmem_base, TMEM_COLS);
     if (threadIdx.x == 32) tstamp(p, MODE, TS_EXIT);
 }
 
@@ -1572,16 +1582,17 @@ static bool make_packed_map(CUtensorMap* m, const void* base, int rows, int cols
 template <int MODE, int NMAX>
 static ms_status launch_gemm(int id, const Maps& maps, const Params& prm, cudaStream_t s) {
     using L = Layout<MODE, NMAX>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE, NMAX>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+    static PerDevice attr;
+    const int ok = attr.get([] {
+        const cudaError_t e =
+            cudaFuncSetAttribute(ffn_gemm_kernel<MODE, NMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
         if (e != cudaSuccess) {
             set_cuda_error(e);
-            return MS_ERR_CUDA;
+            return -1;
         }
-        attr_set = true;
-    }
+        return 1;
+    });
+    if (ok < 0) return MS_ERR_CUDA;
     return launch(id, ffn_gemm_kernel<MODE, NMAX>, dim3(num_sms()), dim3(NTHREADS), L::SMEM, s, maps, prm);
 }
 
@@ -1589,15 +1600,16 @@ static ms_status launch_gemm(int id, const Maps& maps, const Params& prm, cudaSt
 // most one CTA per SM), 0 if the device cannot place any.
 template <int MODE>
 static int pair_grid() {
-    static int grid = -1;
-    if (grid < 0) {
-        grid = 0;
+    // cached per device as grid + 1 (a slot of 0 is empty)
+    static PerDevice cache;
+    return cache.get([]() -> int {
+        int grid = 0;
         if (cudaFuncSetAttribute(ffn_gemm_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  PAIR_SMEM) != cudaSuccess ||
             cudaFuncSetAttribute(ffn_gemm_pair_kernel<MODE>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) !=
                 cudaSuccess) {
             cudaGetLastError();
-            return grid;
+            return grid + 1;
         }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(num_sms());
@@ -1617,8 +1629,8 @@ static int pair_grid() {
         }
         const int cap = num_sms() / 2;
         grid = 2 * (nclusters < cap ? nclusters : cap);
-    }
-    return grid;
+        return grid + 1;
+    }) - 1;
 }
 
 template <int MODE>

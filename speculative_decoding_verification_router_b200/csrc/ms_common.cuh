@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 #include <stdlib.h>
+#include <atomic>
 #include <utility>
 
 #include "moespec.h"
@@ -108,15 +109,49 @@ inline ms_status launch_cluster(int id, void (*kernel)(KArgs...), dim3 grid, dim
     return MS_OK;
 }
 
-inline int num_sms() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
+// ------------------------------------------------------------ per-device host caches
+// Values the host code looks up once per device (SM count, cluster sizes,
+// occupancy) and one-time function attributes (which apply to the device
+// that is current when they are set).  Each cache holds one slot per device,
+// filled by the first call with that device current; the slots are atomics,
+// so two host threads racing on the first fill both compute the same value
+// and neither reads a half-written one.
+constexpr int kMaxDevices = 64;
+
+inline int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        dev = 0;
     }
-    return n;
+    return dev;
+}
+
+// `fill()` must return a non-zero value (0 marks an empty slot).
+struct PerDevice {
+    std::atomic<int> v[kMaxDevices];
+    template <typename F>
+    int get(F fill) {
+        std::atomic<int>& slot = v[current_device()];
+        int x = slot.load(std::memory_order_acquire);
+        if (x == 0) {
+            x = fill();
+            slot.store(x, std::memory_order_release);
+        }
+        return x;
+    }
+};
+
+inline int num_sms() {
+    static PerDevice cache;
+    return cache.get([] {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, current_device()) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 148;
+        }
+        return n;
+    });
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -145,6 +180,14 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Record the first device-side error into a status word (first writer wins).
 __device__ __forceinline__ void report_status(int32_t* status, int32_t code) {
     if (status) atomicCAS(status, 0, code);
+}
+
+// A drain wait (the bounded wait, after a timeout, for a CTA's own loads or
+// MMAs still in flight) ran out as well: recorded over any earlier status,
+// since the CTA now exits with asynchronous work possibly outstanding.
+__device__ __forceinline__ void drain_failed(int32_t* status, volatile int& flag) {
+    if (status) atomicExch(status, MS_ERR_DRAIN_TIMEOUT);
+    flag = 1;
 }
 
 // Warp-wide (value, index) argmax step: larger value wins, equal values go
@@ -194,6 +237,17 @@ __device__ __forceinline__ void st_cluster_s32(const void* local, uint32_t rank,
 // stores above before the loads after it, cluster-wide.
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The value of the same shared-memory int in the other CTA of a pair
+// (after a cluster barrier that orders its last store).
+__device__ __forceinline__ int peer_flag(const volatile int* local) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(const_cast<int*>(local)));
+    uint32_t ra;
+    int v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(cluster_rank() ^ 1u));
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {

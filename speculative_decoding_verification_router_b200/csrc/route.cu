@@ -383,13 +383,13 @@ template <bool NORM>
 static ms_status route_cluster_launch_t(const void* xin, float eps, const float* wr, const float* bias, int T, int H,
                                         int E, int k, int renorm, int32_t* idx, float* w, __nv_bfloat16* xo,
                                         cudaStream_t s) {
-    static bool set = false;
-    if (!set) {
+    static PerDevice set;
+    set.get([] {
         cudaFuncSetAttribute(route_cluster_kernel<NORM, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         cudaFuncSetAttribute(route_cluster_kernel<NORM, RC_TPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              200 * 1024);
-        set = true;
-    }
+        return 1;
+    });
     if (T > 32) {
         const size_t smem = sizeof(float) * static_cast<size_t>(RC_TPC) * (H + E);
         return launch_cluster(K_ROUTE_CLUSTER, route_cluster_kernel<NORM, RC_TPC>,
@@ -420,12 +420,11 @@ ms_status route_launch(const void* x, const float* wr, const float* bias, int T,
     }
     const size_t smem = sizeof(float) * static_cast<size_t>(H + E);
     if (smem > 48 * 1024) {
-        static bool set = false;
-        if (!set) {
-            cudaFuncSetAttribute(route_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 200 * 1024);
-            set = true;
-        }
+        static PerDevice set;
+        set.get([] {
+            cudaFuncSetAttribute(route_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+            return 1;
+        });
     }
     return launch(K_ROUTE_ROWS, route_rows_kernel, dim3(T), dim3(256), smem, s, xb, wr, bias, T,
                   H, E, k, renorm, idx, w);

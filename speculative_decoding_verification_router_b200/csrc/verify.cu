@@ -324,9 +324,9 @@ static bool allow_big_clusters() {
 
 static int verify_cluster_size() {
     // 16-CTA clusters when the device allows them, else the portable 8
-    static int cs = 0;
-    if (cs == 0) {
-        cs = 8;
+    static PerDevice cache;
+    return cache.get([] {
+        int cs = 8;
         if (allow_big_clusters<__nv_bfloat16, 4>() && allow_big_clusters<__nv_bfloat16, 8>() &&
             allow_big_clusters<float, 4>() && allow_big_clusters<float, 8>()) {
             cudaLaunchConfig_t cfg = {};
@@ -345,8 +345,8 @@ static int verify_cluster_size() {
                 cs = 16;
         }
         cudaGetLastError();
-    }
-    return cs;
+        return cs;
+    });
 }
 
 static ms_status verify_cluster_launch(const void* logits, ms_dtype dt, const int32_t* draft, int B, int K, int V,

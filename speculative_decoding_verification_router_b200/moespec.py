@@ -18,7 +18,8 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoespec
 
 MS_F32, MS_BF16 = 0, 1
 STATUS = {0: "MS_OK", -1: "MS_ERR_INVALID_ARG", -2: "MS_ERR_UNSUPPORTED", -3: "MS_ERR_WORKSPACE",
-          -4: "MS_ERR_CUDA", -5: "MS_ERR_TIMEOUT", -6: "MS_ERR_DEVICE_INDEX"}
+          -4: "MS_ERR_CUDA", -5: "MS_ERR_TIMEOUT", -6: "MS_ERR_DEVICE_INDEX",
+          -7: "MS_ERR_DRAIN_TIMEOUT"}
 
 
 class MoeSpecError(RuntimeError):

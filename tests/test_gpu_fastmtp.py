@@ -52,15 +52,28 @@ def test_fastmtp_step_matches_oracle(ms, B, H, I, V):
     d, h = _gpu(ms, w, w["h0"], w["tok0"], K=1)
     rd, rh = _oracle(w, w["h0"], w["tok0"], K=1)
     assert_close(h, rh, what="h after one draft step")
-    # the draft token: equal, or the oracle's logits of the two candidates are within rounding
-    miss = np.nonzero(d[:, 0] != rd[:, 0])[0]
-    if len(miss):
-        _, xb = oracle.rmsnorm(rh)
-        z = oracle.lm_head(oracle.widen_bf16(xb), w["w_lm"])
-        for b in miss:
-            top = z[b, rd[b, 0]]
-            assert top - z[b, d[b, 0]] <= 1e-2 * max(abs(top), 1.0), (b, top, z[b, d[b, 0]])
-    assert len(miss) <= max(1, B // 8)
+    # The draft token is the greedy pick of the vocab head on the step's own
+    # hidden state: every token must be a maximum of the oracle's logits on the
+    # GPU's h (the same head input up to RMSNorm rounding), within the rounding
+    # the GPU applies to them -- the same bound as the fused head's test: one
+    # bf16 rounding of the maximum (2^-7 relative covers both values' rounding)
+    # plus fp32 accumulation over H terms -- and one bf16 ulp (2^-7 relative,
+    # taken at the row's largest |x|) of a head input whose fp32 and fp64
+    # normalisations round apart, times the largest head weight.
+    _, xb = oracle.rmsnorm(h)
+    x = oracle.widen_bf16(xb).astype(np.float64)
+    z = oracle.lm_head(oracle.widen_bf16(xb), w["w_lm"]).astype(np.float64)
+    zmax = z.max(axis=1)
+    zsel = z[np.arange(B), d[:, 0]]
+    wmax = float(np.abs(oracle.widen_bf16(w["w_lm"])).max())
+    tol = np.abs(zmax) * 2.0 ** -7 + 1e-5 * np.sqrt(H) + 2.0 ** -7 * np.abs(x).max(axis=1) * wmax
+    assert np.all(zmax - zsel <= tol), np.nonzero(zmax - zsel > tol)[0]
+    # and on the oracle's own hidden state the picks agree except where two
+    # candidates lie within that bound of each other (a near-tie)
+    zr = oracle.lm_head(oracle.widen_bf16(oracle.rmsnorm(rh)[1]), w["w_lm"]).astype(np.float64)
+    for b in np.nonzero(d[:, 0] != rd[:, 0])[0]:
+        gap = zr[b, rd[b, 0]] - zr[b, d[b, 0]]
+        assert gap <= tol[b] + 2 * np.abs(z[b] - zr[b]).max(), (b, gap)
 
 
 def test_fastmtp_recursion_equals_chained_steps(ms):
