@@ -6,6 +6,7 @@
 #include <vector>
 
 #include "ms_common.cuh"
+#include "layer_fused.cuh"
 
 namespace ms {
 
@@ -29,7 +30,7 @@ static const char* kNames[K_COUNT] = {
     "rmsnorm",        "route_rows",      "route_tiled",     "route_cluster", "permute_count", "permute_scatter",
     "ffn_prep",       "gemm1_stream",    "gemm2_stream",    "gemm1_tiled",   "gemm2_tiled",  "ffn_finish",
     "lm_head_stream", "combine",         "verify_partial",  "verify_final",  "verify_cluster", "verify_keys", "wait_probe",
-    "pack_weights",   "mtp_prep"};
+    "pack_weights",   "mtp_prep",        "moe_stream_layer"};
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kNames[id] : "?"; }
 
@@ -99,7 +100,7 @@ __global__ void wait_probe_kernel(const int32_t* flag, int32_t expect, int32_t* 
 struct LayerWs {
     void* xhat;
     int32_t *idx, *offsets, *perm, *slot;
-    float *w, *y_perm, *y_sh;
+    float *w, *y_perm, *y_sh, *logits;
     void *perm_ws, *ffn_ws;
     size_t perm_bytes, ffn_bytes, bytes;
 };
@@ -126,6 +127,7 @@ static LayerWs layer_layout(void* base, int T, int H, int E, int I, int S, int k
     w.perm_ws = take(w.perm_bytes);
     w.y_perm = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * H * (T <= 128 ? 4 : 2)));
     w.y_sh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * H * 4));
+    w.logits = reinterpret_cast<float*>(take(static_cast<size_t>(T) * E * 4));
     w.bytes = off;
     return w;
 }
@@ -154,11 +156,28 @@ ms_status moe_layer_forward(const float* a, const float* w_router, const float* 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const ms_dtype ydt = T <= 128 ? MS_F32 : MS_BF16;
     int32_t* status = static_cast<int32_t*>(w.ffn_ws);
-    // the status word reports this call's device-side conditions only
-    cudaError_t ce = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+    // The status word reports this call's device-side conditions only; the
+    // fused kernel's grid-barrier counter shares its 256-byte block.
+    cudaError_t ce = cudaMemsetAsync(status, 0, 256, s);
     if (ce != cudaSuccess) {
         ms::set_cuda_error(ce);
         return MS_ERR_CUDA;
+    }
+    if (ms::layer_fused_supported(T, H, E, I, S, k)) {
+        // verify-sized batch: the whole layer in one persistent kernel
+        ms::LfBuffers b{};
+        ms::ffn_ws_buffers(w.ffn_ws, T, H, E, I, S, k, b);
+        b.logits = w.logits;
+        b.y_perm = w.y_perm;
+        b.y_sh = w.y_sh;
+        b.idx = w.idx;
+        b.off = w.offsets;
+        b.perm = w.perm;
+        b.slot = w.slot;
+        b.w = w.w;
+        b.bar = reinterpret_cast<unsigned int*>(static_cast<char*>(w.ffn_ws) + 128);
+        return ms::layer_fused_launch(a, w_router, logit_bias, w_gate_up, w_down, ws_gate_up, ws_down, T, H, E, I, S,
+                                      k, renormalize, 1e-6f, out, b, s);
     }
     ms_status st;
     if (T < 1024) {

@@ -28,6 +28,7 @@
 // Shared experts form one extra group whose intermediate width is S*I: two
 // SwiGLU experts equal one expert with the intermediates concatenated.
 #include "ffn_core.cuh"
+#include "layer_fused.cuh"
 
 namespace ms {
 
@@ -1030,6 +1031,18 @@ static FfnWs ffn_ws_layout(void* base, int T, int H, int E, int I, int S, int k)
 
 size_t ffn_ws_bytes(int T, int H, int E, int I, int S, int k) {
     return ffn_ws_layout(nullptr, T, H, E, I, S, k).bytes;
+}
+
+void ffn_ws_buffers(void* ws, int T, int H, int E, int I, int S, int k, LfBuffers& b) {
+    const FfnWs w = ffn_ws_layout(ws, T, H, E, I, S, k);
+    b.x_pad = w.x_pad;
+    b.x_perm = w.x_perm;
+    b.h_perm = w.h_perm;
+    b.h_sh = w.h_sh;
+    b.partials = w.partials;
+    b.status = w.status;
+    b.rows_pad = w.rows_pad;
+    b.t_pad = w.t_pad;
 }
 
 ms_status ffn_launch(const void* x, const int32_t* offsets, const int32_t* perm, const void* wgu,

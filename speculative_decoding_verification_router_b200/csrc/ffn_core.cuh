@@ -143,6 +143,7 @@ __device__ __forceinline__ void warp_scan_groups(int* a, int n, int lane) {
 // largest g with tprefix[g] <= t
 __device__ __forceinline__ int find_group_tile(const Sched& s, int t) {
     int lo = 0, hi = s.ngroups - 1;
+#pragma unroll 1
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (s.tprefix[mid] <= t) lo = mid; else hi = mid - 1;
@@ -194,11 +195,18 @@ __device__ __forceinline__ int step_cost(const Sched& s, int g) {
 // token-operand rows and its first row; build_schedule_n reads them from the
 // routing offsets in global memory, the fused layer kernel from its own
 // shared-memory copy.
-template <int MODE, int NT, typename GroupRows>
-__device__ void build_schedule_g(const Params& p, Sched& s, int ngroups, GroupRows group_rows) {
-    const int tid = threadIdx.x;
+// NT threads build it, thread `tid` = 0..NT-1 of them (every thread of the
+// CTA must call it: it contains CTA barriers).
+struct CtaSync {
+    __device__ void operator()() const { __syncthreads(); }
+};
+
+template <int MODE, int NT, typename GroupRows, typename Sync = CtaSync>
+__device__ void build_schedule_g(const Params& p, Sched& s, int ngroups, GroupRows group_rows,
+                                 int tid = static_cast<int>(threadIdx.x), Sync sync = Sync()) {
     s.ngroups = ngroups;
     const int ng = s.ngroups;
+#pragma unroll 1
     for (int g = tid; g < ng; g += NT) {
         int rows, row0;
         group_rows(g, rows, row0);
@@ -218,11 +226,11 @@ __device__ void build_schedule_g(const Params& p, Sched& s, int ngroups, GroupRo
         s.tprefix[g + 1] = tiles;
         if (Cfg<MODE>::kStream) s.fcp[g + 1] = units * step_cost<MODE>(s, g);
     }
-    __syncthreads();
+    sync();
     if (tid < 32) warp_scan_groups(s.prefix, ng, tid);
     else if (tid < 64) warp_scan_groups(s.tprefix, ng, tid - 32);
     else if (Cfg<MODE>::kStream && tid < 96) warp_scan_groups(s.fcp, ng, tid - 64);
-    __syncthreads();
+    sync();
     if (Cfg<MODE>::kStream) {
         // the split region: the tiles after the nct * D whole tiles
         __shared__ int skb_cost;   // cost of the k-steps before the split region
@@ -238,7 +246,7 @@ __device__ void build_schedule_g(const Params& p, Sched& s, int ngroups, GroupRo
             s.sk_begin = skb;
             skb_cost = cskb;
         }
-        __syncthreads();
+        sync();
         // CTA c's range starts at the first k-step whose cost from the start
         // of the split region reaches c/nct of the region's cost
         const int nct = p.nct, total = s.prefix[ng];
@@ -246,6 +254,7 @@ __device__ void build_schedule_g(const Params& p, Sched& s, int ngroups, GroupRo
         // 32-bit arithmetic when the scaled costs fit (every layer of this
         // model); 64-bit division is several times slower
         const bool narrow = static_cast<long long>(s.fcp[ng]) * nct < (1LL << 31);
+#pragma unroll 1
         for (int c = tid; c <= nct; c += NT) {
             int b;
             if (c == 0 || C == 0) {
@@ -255,6 +264,7 @@ __device__ void build_schedule_g(const Params& p, Sched& s, int ngroups, GroupRo
             } else {
                 const long long x = C * c + C0 * nct;   // the target cost, times nct
                 int lo = 0, hi = ng - 1;                // largest g with fcp[g] * nct <= x
+#pragma unroll 1
                 while (lo < hi) {
                     const int mid = (lo + hi + 1) >> 1;
                     if (static_cast<long long>(s.fcp[mid]) * nct <= x) lo = mid; else hi = mid - 1;
@@ -268,7 +278,7 @@ __device__ void build_schedule_g(const Params& p, Sched& s, int ngroups, GroupRo
             }
             s.rb[c] = b;
         }
-        __syncthreads();
+        sync();
     }
 }
 

@@ -36,6 +36,7 @@ enum KernelId : int {
     K_WAIT_PROBE,
     K_PACK,
     K_MTP_PREP,
+    K_LAYER_FUSED,
     K_COUNT
 };
 const char* kernel_name(int id);

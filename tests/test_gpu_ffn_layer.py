@@ -259,8 +259,22 @@ def test_trace_records_kernels(ms):
         ms.trace_disable()
         ms.trace_reset()
     names = [n for n, _ in recs]
-    assert names == ["route_cluster", "permute_scatter", "ffn_prep", "gemm1_stream", "ffn_finish", "gemm2_stream",
-                     "ffn_finish", "combine"], names
+    # a layer of at most 16 tokens is one persistent launch (routing, both GEMMs, their sums, combine)
+    assert names == ["moe_stream_layer"], names
+    # more tokens: the chain of launches
+    shp32 = synth.VERIFY_B32
+    a32, lw32, b32 = routed_layer_inputs(shp32, 0)
+    w32 = _weights_dev(lw32)
+    ms.trace_enable(64)
+    try:
+        ms.layer_forward(dev(a32), dev(lw32.w_router), dev(b32), *w32, shp32.k)
+        torch.cuda.synchronize()
+        names32 = [n for n, _ in ms.trace_records()]
+    finally:
+        ms.trace_disable()
+        ms.trace_reset()
+    assert names32 == ["route_cluster", "permute_scatter", "ffn_prep", "gemm1_stream", "ffn_finish", "gemm2_stream",
+                       "ffn_finish", "combine"], names32
     assert all(t > 0 for _, t in recs)
 
 
