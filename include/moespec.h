@@ -274,6 +274,26 @@ MS_API ms_status moe_layer_forward(const float* a, const float* w_router, const 
  * and clears it. */
 MS_API ms_status ms_device_status(void* ws, void* stream);
 
+/* Batch-invariant schedules (default off).  The pages call speculative
+ * greedy decoding lossless: the tokens it commits are byte-identical to plain
+ * greedy decoding (the d9249 blog, "핵심 아이디어 / 구조 / 동작 방식";
+ * clawpit.io, "Speculative decoding without accuracy loss").  That holds
+ * exactly only if a position's logits do not depend on how many other
+ * positions share its forward pass -- K+1 verify rows versus one greedy row.
+ * By default the weight-streaming GEMMs (moe_expert_ffn and the layer at
+ * T <= 128, lm_head_logits, spec_verify_lm_head_greedy, fastmtp_draft) split
+ * output tiles between CTAs at points that depend on the batch, so the last
+ * bit of a sum may change with it.  With this setting on, every call issued
+ * afterwards (process-wide) computes each output tile whole in one CTA with
+ * k in natural order, and moe_layer_forward does not use its fused
+ * small-batch kernel: every token's results are then bit-identical whatever
+ * else is in the batch (the routing, normalisation, combine and verify are
+ * per-token already).  Cost: the tiles are dealt round-robin, without the
+ * split that balances them over the SMs.  The prefill-sized (T > 128) tiled
+ * path computes each token row whole in any case, in an order of its own. */
+MS_API void ms_set_batch_invariant(int on);
+MS_API int ms_get_batch_invariant(void);
+
 /* Bounded-wait limit used by every device-side spin (default 1e9 ns). */
 MS_API void ms_set_wait_limit_ns(uint64_t ns);
 MS_API uint64_t ms_get_wait_limit_ns(void);

@@ -2,6 +2,7 @@
 // self-test, launch tracing, the whole-layer composite, version/strings.
 #include <stdio.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -43,6 +44,10 @@ void set_cuda_error(cudaError_t e) {
 // ------------------------------------------------------------ wait limit
 static uint64_t g_wait_limit_ns = 1000000000ull;
 uint64_t wait_limit_ns() { return g_wait_limit_ns; }
+
+// ------------------------------------------------------------ batch-invariant schedules
+static std::atomic<int> g_batch_invariant{0};
+int batch_invariant() { return g_batch_invariant.load(std::memory_order_relaxed); }
 
 // ------------------------------------------------------------ tracing
 struct TraceRec {
@@ -163,7 +168,7 @@ ms_status moe_layer_forward(const float* a, const float* w_router, const float* 
         ms::set_cuda_error(ce);
         return MS_ERR_CUDA;
     }
-    if (ms::layer_fused_supported(T, H, E, I, S, k)) {
+    if (!ms::batch_invariant() && ms::layer_fused_supported(T, H, E, I, S, k)) {
         // verify-sized batch: the whole layer in one persistent kernel
         ms::LfBuffers b{};
         ms::ffn_ws_buffers(w.ffn_ws, T, H, E, I, S, k, b);
@@ -217,6 +222,9 @@ ms_status ms_device_status(void* ws, void* stream) {
 }
 
 void ms_set_wait_limit_ns(uint64_t ns) { ms::g_wait_limit_ns = ns; }
+
+void ms_set_batch_invariant(int on) { ms::g_batch_invariant.store(on ? 1 : 0, std::memory_order_relaxed); }
+int ms_get_batch_invariant(void) { return ms::batch_invariant(); }
 
 ms_status ms_set_device_trace(void* buf, size_t bytes) {
     if (buf && bytes < static_cast<size_t>(8) * 256 * 8 * sizeof(uint64_t)) return MS_ERR_WORKSPACE;

@@ -960,8 +960,10 @@ static ms_status launch_stream_n(int id, const Maps& maps, Params prm, cudaStrea
     prm.nct = num_sms();
     if (prm.nct > MAX_CTAS) return MS_ERR_UNSUPPORTED;   // the schedule keeps one range per CTA
     prm.weights_evict_first = evict_first_allowed();
+    prm.invariant = batch_invariant();
     ms_status st = launch_gemm<MODE, NMAX>(id, maps, prm, s);
     if (st != MS_OK) return st;
+    if (prm.invariant) return MS_OK;   // every tile whole: no split tiles to finish
     // fewer than 2 nct tiles are split; one CTA per (tile, 16-column chunk)
     return launch(K_FFN_FINISH, ffn_finish_kernel<MODE, NMAX>, dim3(finish_grid<MODE, NMAX>(prm.nct)),
                   dim3(FIN_THREADS), 0, s, prm);

@@ -60,6 +60,7 @@ struct Params {
     float* partials;               // 2 partial-sum slots per CTA (streaming)
     int nct;                       // grid size of the streaming GEMM (for the finish kernel)
     int weights_evict_first;       // streaming: weight tiles are loaded with an L2 evict-first policy
+    int invariant;                 // streaming: batch-invariant schedule (whole tiles, natural k order)
     int32_t* status;
     uint64_t wait_limit_ns;
     uint64_t* dtrace;              // optional per-CTA timeline (see ms_set_device_trace)
@@ -364,7 +365,8 @@ struct WorkIter {
     // partials; the finish kernel that follows the GEMM sums them and applies
     // the epilogue.
     // Tiled: tiles c, c + nct, ... (round robin).
-    int c, nct, state, pos, re, dp_next, dp_end, t, total;
+    int c, nct, state, pos, re, dp_next, dp_end, dp_step, t, total;
+    bool rotate;
     const Sched* sp;
 
     __device__ void init(const Params& p, const Sched& s, int c_, int nct_) {
@@ -377,9 +379,21 @@ struct WorkIter {
             const int D = dp_tiles_per_cta(nt, nct);
             dp_next = c * D;
             dp_end = dp_next + D;
+            dp_step = 1;
+            rotate = true;
             pos = sk_range_begin(c);
             re = sk_range_begin(c + 1);
             state = 0;
+            if (p.invariant) {
+                // batch-invariant: tiles c, c + nct, ... each whole, k in natural
+                // order -- an output's sum does not depend on the other tokens
+                dp_next = c;
+                dp_end = nt;
+                dp_step = nct;
+                rotate = false;
+                pos = re = 0;
+                state = 1;
+            }
         } else {
             t = c;
         }
@@ -425,8 +439,8 @@ struct WorkIter {
                 w.kt = group_ktiles<MODE>(p, g);
                 w.k1 = w.kt;
                 w.tile_start = s.prefix[g] + w.n * w.kt;
-                w.rot = c % w.kt;
-                ++dp_next;
+                w.rot = rotate ? c % w.kt : 0;
+                dp_next += dp_step;
                 return true;
             }
             return false;

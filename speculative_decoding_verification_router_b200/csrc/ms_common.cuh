@@ -44,6 +44,7 @@ const char* kernel_name(int id);
 // ------------------------------------------------------------ host side
 void trace_mark(int id, cudaStream_t s, bool after);
 uint64_t wait_limit_ns();
+int batch_invariant();
 void set_cuda_error(cudaError_t e);
 
 // Programmatic dependent launch is on unless MOESPEC_NO_PDL=1 (a measurement

@@ -69,6 +69,8 @@ def _load():
         "ms_version": (I, []),
         "moe_pack_weights": (I, [P, I, I, I, P, P]),
         "ms_set_device_trace": (I, [P, Z]),
+        "ms_set_batch_invariant": (None, [I]),
+        "ms_get_batch_invariant": (I, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -342,6 +344,16 @@ def layer_forward(a, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down, k: 
 def device_status(ws: Workspace, stream=None) -> int:
     """Synchronise, return and clear the device status word kept in `ws`."""
     return int(_lib.ms_device_status(ws.c(), _stream(stream)))
+
+
+def set_batch_invariant(on: bool):
+    """Process-wide: batch-invariant GEMM schedules for the calls that follow
+    (see ms_set_batch_invariant in include/moespec.h)."""
+    _lib.ms_set_batch_invariant(int(bool(on)))
+
+
+def get_batch_invariant() -> bool:
+    return bool(_lib.ms_get_batch_invariant())
 
 
 def set_wait_limit_ns(ns: int):

@@ -106,3 +106,17 @@ def test_product_path_never_imports_the_oracle():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "moe_oracle" not in txt, f
+
+
+def test_batch_invariant_setting_round_trips(lib):
+    # a host-side switch: no GPU needed to set and read it
+    lib.ms_get_batch_invariant.restype = ctypes.c_int
+    lib.ms_set_batch_invariant.argtypes = [ctypes.c_int]
+    old = lib.ms_get_batch_invariant()
+    try:
+        lib.ms_set_batch_invariant(1)
+        assert lib.ms_get_batch_invariant() == 1
+        lib.ms_set_batch_invariant(0)
+        assert lib.ms_get_batch_invariant() == 0
+    finally:
+        lib.ms_set_batch_invariant(old)
