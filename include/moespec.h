@@ -92,6 +92,22 @@ MS_API ms_status moe_route_topk(const void* xhat, const float* w_router, const f
                          int T, int H, int E, int k, int renormalize,
                          int32_t* topk_idx, float* topk_w, void* stream);
 
+/* a1 on the tensor cores, for prefill-sized batches: the same results as
+ * moe_route_topk (same ordering and tie rule; gate weights equal up to fp32
+ * rounding) from a tcgen05 GEMM.  W_r is split into three bf16 parts
+ * hi + mid + lo that carry its fp32 significand (each part's rounding error is
+ * exact in fp32), so xhat . W_r = (xhat . hi + xhat . mid) + xhat . lo with
+ * exact bf16 products and fp32 accumulation: the logits agree with the fp32
+ * ones to within fp32 rounding of the sums.  Softmax and top-k run in the
+ * GEMM's epilogue.  E % 16 == 0, E <= 64, k <= 8, H % 128 == 0.
+ * Scratch: moe_route_topk_tensor_workspace_size(E, H) bytes (a status word
+ * and the split weights); moe_layer_forward uses this form for T >= 1024. */
+MS_API size_t moe_route_topk_tensor_workspace_size(int E, int H);
+MS_API ms_status moe_route_topk_tensor(const void* xhat, const float* w_router, const float* logit_bias,
+                                       int T, int H, int E, int k, int renormalize,
+                                       int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                                       void* stream);
+
 /* a2  Permutation: group the T*k (token, slot) pairs by expert, ordered by
  * (expert, token) -- a stable counting sort, bit-exact and deterministic.
  * expert_offsets: [E+1] int32, expert e owns rows [off[e], off[e+1]).

@@ -21,6 +21,10 @@ size_t permute_ws_bytes(int, int, int);
 ms_status permute_launch(const int32_t*, int, int, int, int32_t*, int32_t*, int32_t*, void*, int32_t*,
                          cudaStream_t);
 size_t ffn_ws_bytes(int, int, int, int, int, int);
+size_t route_tc_ws_bytes(int, int);
+bool route_tc_supported(int, int, int);
+ms_status route_tc_launch(const void*, const float*, const float*, int, int, int, int, int, int32_t*, float*, void*,
+                          int32_t*, cudaStream_t);
 ms_status ffn_launch(const void*, const int32_t*, const int32_t*, const void*, const void*, const void*,
                      const void*, int, int, int, int, int, int, void*, ms_dtype, float*, void*, cudaStream_t);
 ms_status combine_launch(const void*, ms_dtype, const float*, const int32_t*, const float*, const float*,
@@ -31,7 +35,7 @@ static const char* kNames[K_COUNT] = {
     "rmsnorm",        "route_rows",      "route_tiled",     "route_cluster", "permute_count", "permute_scatter",
     "ffn_prep",       "gemm1_stream",    "gemm2_stream",    "gemm1_tiled",   "gemm2_tiled",  "ffn_finish",
     "lm_head_stream", "combine",         "verify_partial",  "verify_final",  "verify_cluster", "verify_keys", "wait_probe",
-    "pack_weights",   "mtp_prep",        "moe_stream_layer"};
+    "pack_weights",   "mtp_prep",        "moe_stream_layer", "route_tc",     "route_split"};
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kNames[id] : "?"; }
 
@@ -106,7 +110,7 @@ struct LayerWs {
     void* xhat;
     int32_t *idx, *offsets, *perm, *slot;
     float *w, *y_perm, *y_sh, *logits;
-    void *perm_ws, *ffn_ws;
+    void *perm_ws, *ffn_ws, *route_ws;
     size_t perm_bytes, ffn_bytes, bytes;
 };
 
@@ -133,6 +137,7 @@ static LayerWs layer_layout(void* base, int T, int H, int E, int I, int S, int k
     w.y_perm = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * H * (T <= 128 ? 4 : 2)));
     w.y_sh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * H * 4));
     w.logits = reinterpret_cast<float*>(take(static_cast<size_t>(T) * E * 4));
+    w.route_ws = T >= 1024 ? take(route_tc_ws_bytes(E, H)) : nullptr;   // the split router weights
     w.bytes = off;
     return w;
 }
@@ -191,7 +196,12 @@ ms_status moe_layer_forward(const float* a, const float* w_router, const float* 
                                       w.xhat, s);
     } else {
         st = ms::rmsnorm_launch(a, nullptr, T, H, 1e-6f, w.xhat, s);
-        if (st == MS_OK)
+        // prefill-sized: the router on the tensor cores (B200: 281 -> ~20 us at
+        // 36,992 tokens) where the shape allows, else the fp32 CUDA-core router
+        if (st == MS_OK && ms::route_tc_supported(E, k, H))
+            st = ms::route_tc_launch(w.xhat, w_router, logit_bias, T, H, E, k, renormalize, w.idx, w.w, w.route_ws,
+                                     status, s);
+        else if (st == MS_OK)
             st = ms::route_launch(w.xhat, w_router, logit_bias, T, H, E, k, renormalize, w.idx, w.w, s);
     }
     if (st == MS_OK) st = ms::permute_launch(w.idx, T, k, E, w.offsets, w.perm, w.slot, w.perm_ws, status, s);

@@ -30,14 +30,108 @@
 #include "ffn_core.cuh"
 #include "layer_fused.cuh"
 
+#include <algorithm>
+
 namespace ms {
 
 using namespace sm100;
 
+// ------------------------------------------------------------ router epilogue
+// Softmax over the E logits of token t and its k largest (larger logit first,
+// equal logits to the lower expert), in registers: one pass keeps the k best in
+// descending order.  Gate weight = softmax probability, divided by the sum of
+// the k chosen when renormalising.
+constexpr int ROUTE_TC_EMAX = 64;
+constexpr int ROUTE_TC_KMAX = 8;
+
+// The router's epilogue for one token row (this thread's TMEM lane), in
+// registers only: in this kernel shared memory takes nearly all of L1, so a
+// per-thread array indexed at run time would live in L2.  Two passes over the
+// logits in chunks of 16, reloaded from TMEM: the maximum and the 8 best (kept
+// in descending order, a later expert never passing an equal earlier one; the
+// first k are the top-k), then the softmax denominator.  Every lane executes the TMEM
+// loads (warp-collective); only a valid row stores.
+template <typename TmemAt>
+__device__ __forceinline__ void route_chunk(const Params& p, TmemAt tmem_at, int c16, int t, bool valid,
+                                            float (&z)[16]) {
+    float h16[16], m16[16], l16[16];
+    tmem_ld16(tmem_at(c16 * 16), h16);
+    tmem_ld16(tmem_at(p.E + c16 * 16), m16);
+    tmem_ld16(tmem_at(2 * p.E + c16 * 16), l16);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) z[j] = (h16[j] + m16[j]) + l16[j];
+    if (p.rbias && valid) {
+        const float* b = p.rbias + static_cast<size_t>(t) * p.E + c16 * 16;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) z[j] += __ldg(b + j);
+    }
+}
+
+template <typename TmemAt>
+__device__ __forceinline__ void route_epilogue(const Params& p, TmemAt tmem_at, int t, bool valid) {
+    const int E = p.E, k = p.k;
+    float tv[ROUTE_TC_KMAX];   // the 8 best so far, descending (ti < 0: empty); the first k are the top-k
+    int ti[ROUTE_TC_KMAX];
+#pragma unroll
+    for (int j = 0; j < ROUTE_TC_KMAX; ++j) {
+        tv[j] = -INFINITY;
+        ti[j] = -1;
+    }
+    float m = -INFINITY;
+#pragma unroll 1
+    for (int c16 = 0; c16 * 16 < E; ++c16) {
+        float z[16];
+        route_chunk(p, tmem_at, c16, t, valid, z);
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+            m = fmaxf(m, z[jj]);
+            // bubble (z, e) into the list of the 8 best, ordered by logit
+            // descending, then expert ascending: at each place the first of
+            // the carried and the held entry in that order stays (a displaced
+            // entry carries on with the same comparison)
+            float cv = z[jj];
+            int ci = c16 * 16 + jj;
+#pragma unroll
+            for (int j = 0; j < ROUTE_TC_KMAX; ++j) {
+                const bool take = ti[j] < 0 || cv > tv[j] || (cv == tv[j] && ci < ti[j]);
+                const float hv = tv[j];
+                const int hi = ti[j];
+                tv[j] = take ? cv : hv;
+                ti[j] = take ? ci : hi;
+                cv = take ? hv : cv;
+                ci = take ? hi : ci;
+            }
+        }
+    }
+    float s = 0.f;
+#pragma unroll 1
+    for (int c16 = 0; c16 * 16 < E; ++c16) {
+        float z[16];
+        route_chunk(p, tmem_at, c16, t, valid, z);
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) s += expf(z[jj] - m);
+    }
+    if (!valid) return;
+    float psum = 0.f;
+#pragma unroll
+    for (int j = 0; j < ROUTE_TC_KMAX; ++j)
+        if (j < k) {
+            tv[j] = expf(tv[j] - m) / s;
+            psum += tv[j];
+        }
+#pragma unroll
+    for (int j = 0; j < ROUTE_TC_KMAX; ++j)
+        if (j < k) {
+            p.ridx[static_cast<size_t>(t) * k + j] = ti[j];
+            p.rw[static_cast<size_t>(t) * k + j] = p.rrenorm ? tv[j] / psum : tv[j];
+        }
+}
+
 // ------------------------------------------------------------ kernel
 template <int MODE, int NMAX>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
+    ffn_gemm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
     using L = Layout<MODE, NMAX>;
     constexpr bool kStream = Cfg<MODE>::kStream;
     constexpr int kSub = Cfg<MODE>::kSub;
@@ -126,6 +220,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int sb = 0; sb < kSub; ++sb)
                 ld(a + sb * TILE_BYTES, &maps.w_a, packed_row(w.n * BM, kt * kSub + sb, kt_h), 0);
+        } else if (MODE == ROUTE_TILED) {
+            // the three bf16 parts of the router weights, [3E][H] row-major: k offset in x
+            tma_load_3d(b, &maps.w_a, full, kx, 0, 0);
         } else {   // G2_TILED
             const int n0 = w.n * p.bn;
             for (int j = 0; j < p.bn / BM; ++j) {
@@ -140,7 +237,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     };
     auto weight_bytes = [&]() -> uint32_t {
         if (MODE == G1_STREAM || MODE == G1_TILED) return 2 * TILE_BYTES;
-        if (MODE == G2_TILED) return p.bn * BK * 2;
+        if (MODE == G2_TILED || MODE == ROUTE_TILED) return p.bn * BK * 2;
         return kSub * TILE_BYTES;
     };
     auto token_loads = [&](const Work& w, int kt, uint32_t a, uint32_t b, uint32_t full) -> uint32_t {
@@ -167,11 +264,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // Weight tiles do not depend on the previous kernel: start streaming
         // the first stages now, while it drains.  (Prefetching further
         // k-steps into L2 as well measured slower: the extra requests delay
-        // the ones the pipeline waits for.)
+        // the ones the pipeline waits for.)  The router's split weights are
+        // the exception: the launch just before writes them.
         WorkIter<MODE> it;
         it.init(p, sched, c, nct);
         Work w;
-        while (npre < ST && it.next(p, sched, w)) {
+        while (MODE != ROUTE_TILED && npre < ST && it.next(p, sched, w)) {
             for (int i = w.k0; i < w.k1 && npre < ST; ++i, ++npre) {
                 const uint32_t a = sbase + npre * L::STAGE, full = smem_addr(&bar_full[npre]);
                 mbar_expect_tx_only(full, weight_bytes());
@@ -232,8 +330,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int q_end = q_issued > npre ? q_issued : npre;
         for (int s2 = 0; s2 < ST && s2 < q_end; ++s2) {
             const int q_last = s2 + ((q_end - 1 - s2) / ST) * ST;
-            volatile int never = 0;
-            if (!mbar_wait(smem_addr(&bar_full[s2]), static_cast<uint32_t>(q_last / ST) & 1u, lim, &never))
+            if (!mbar_wait(smem_addr(&bar_full[s2]), static_cast<uint32_t>(q_last / ST) & 1u, lim, nullptr))
                 drain_failed(p.status, drain_fail_sh);
         }
         tstamp(p, MODE, TS_PRODUCER_DONE);
@@ -297,8 +394,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tstamp(p, MODE, TS_LAST_MMA);
         // drain: all MMAs issued by this thread complete before TMEM is freed
         mma_commit(smem_addr(&bar_drain));
-        volatile int never = 0;
-        if (!mbar_wait(smem_addr(&bar_drain), 0, lim, &never)) drain_failed(p.status, drain_fail_sh);
+        if (!mbar_wait(smem_addr(&bar_drain), 0, lim, nullptr)) drain_failed(p.status, drain_fail_sh);
       }
       __syncwarp();
     } else {
@@ -397,7 +493,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int rr = w.m0 + r_in;                  // row within the group
                 const bool valid = rr < rows;
                 const size_t orow = static_cast<size_t>(shared ? rr : row0 + rr);
-                if (MODE == G1_TILED) {
+                if (MODE == ROUTE_TILED) {
+                    // logit of expert e = (hi + mid) + lo parts, columns e, E + e, 2E + e
+                    route_epilogue(p, tmem_at, rr, valid);
+                } else if (MODE == G1_TILED) {
                     const int f0 = w.n * BM;
                     __nv_bfloat16* dst = shared ? p.h_sh + orow * ldh_s + f0 : p.h_perm + orow * ldh_r + f0;
                     for (int ch = 0; ch < BM / 16; ++ch) {
@@ -485,7 +584,7 @@ constexpr int PAIR_SMEM = PAIR_ST * PAIR_STAGE + 1024;
 
 template <int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    ffn_gemm_pair_kernel(const __grid_constant__ Maps maps, const Params p) {
+    ffn_gemm_pair_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
     static_assert(MODE == G1_TILED || MODE == G2_TILED, "CTA pairs run the tiled schedule");
     constexpr int ST = PAIR_ST;
     extern __shared__ uint8_t dsmem[];
@@ -588,8 +687,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // released its stage (they waited for the full pair of loads)
         for (int s2 = 0; s2 < ST && s2 < q; ++s2) {
             const int q_last = s2 + ((q - 1 - s2) / ST) * ST;
-            volatile int never = 0;
-            if (!mbar_wait(smem_addr(&bar_empty[s2]), static_cast<uint32_t>(q_last / ST) & 1u, lim, &never))
+            if (!mbar_wait(smem_addr(&bar_empty[s2]), static_cast<uint32_t>(q_last / ST) & 1u, lim, nullptr))
                 drain_failed(p.status, drain_fail_sh);
         }
         tstamp(p, MODE, TS_PRODUCER_DONE);
@@ -645,8 +743,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tstamp(p, MODE, TS_LAST_MMA);
             // drain: every pair MMA issued by this thread completes before TMEM is freed
             mma_commit_pair(mapa_shared(smem_addr(&bar_drain), 0));
-            volatile int never = 0;
-            if (!mbar_wait(smem_addr(&bar_drain), 0, lim, &never)) drain_failed(p.status, drain_fail_sh);
+            if (!mbar_wait(smem_addr(&bar_drain), 0, lim, nullptr)) drain_failed(p.status, drain_fail_sh);
         }
       }
       __syncwarp();
@@ -750,7 +847,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 template <int MODE, int NMAX>
-__global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const Params p) {
+__global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const __grid_constant__ Params p) {
     __shared__ Sched sched;
     __shared__ int iprefix[MAX_GROUPS + 1];   // items before group g
     fin_stamp<MODE>(p, TS_ENTRY);
@@ -1167,6 +1264,63 @@ ms_status lm_launch(const void* x, const void* wlm, int T, int H, int V, void* l
     return MS_OK;
 }
 
+// ------------------------------------------------------------ router on the tensor cores
+// W_r (fp32) as three bf16 parts hi + mid + lo: hi = bf16(w), mid = bf16(w - hi),
+// lo = bf16(w - hi - mid) -- each difference is exact in fp32, and the three
+// parts carry the 24-bit significand.  Rows [s][E][H], s = 0, 1, 2.
+__global__ void __launch_bounds__(256) route_split_kernel(const float* __restrict__ wr, int n,
+                                                          __nv_bfloat16* __restrict__ w3) {
+    grid_dep_wait();
+    grid_dep_launch();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const float w = __ldg(wr + i);
+        const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+        const float r1 = w - __bfloat162float(hi);
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(mid);
+        w3[i] = hi;
+        w3[n + i] = mid;
+        w3[2 * n + i] = __float2bfloat16_rn(r2);
+    }
+}
+
+size_t route_tc_ws_bytes(int E, int H) { return align_up(256, 1024) + align_up(static_cast<size_t>(3) * E * H * 2, 1024); }
+
+bool route_tc_supported(int E, int k, int H) {
+    return E % 16 == 0 && E <= ROUTE_TC_EMAX && k <= ROUTE_TC_KMAX && H % BK == 0;
+}
+
+// logits = xhat [T][H] (bf16) . W_r^T as (xhat . hi^T + xhat . mid^T) + xhat . lo^T
+// with exact bf16 products and fp32 accumulation on the tensor cores, 128
+// tokens per tile (tiles dealt round-robin to one CTA per SM); softmax and
+// top-k in the epilogue.  ws: status word + the split weights.
+ms_status route_tc_launch(const void* x, const float* wr, const float* bias, int T, int H, int E, int k, int renorm,
+                          int32_t* idx, float* w, void* ws, int32_t* status, cudaStream_t s) {
+    char* base = static_cast<char*>(ws);
+    auto* w3 = reinterpret_cast<__nv_bfloat16*>(base + align_up(256, 1024));
+    const int n = E * H;
+    ms_status st = launch(K_ROUTE_SPLIT, route_split_kernel, dim3(std::min((n + 255) / 256, 2 * num_sms())),
+                          dim3(256), 0, s, wr, n, w3);
+    if (st != MS_OK) return st;
+    Maps m{};
+    if (!make_map(&m.w_a, w3, H, 3 * E, 1, 3 * E) || !make_map(&m.tok_r, x, H, T, 1, BM)) return MS_ERR_CUDA;
+    m.w_s = m.w_a;
+    m.tok_s = m.tok_r;
+    Params prm{};
+    prm.T = T; prm.H = H; prm.E = E; prm.I = BM; prm.S = 0; prm.k = k; prm.V = 0;
+    prm.bn = 3 * E;
+    prm.offsets = nullptr;
+    prm.rbias = bias;
+    prm.ridx = idx;
+    prm.rw = w;
+    prm.rrenorm = renorm;
+    prm.nct = num_sms();
+    prm.status = status ? status : reinterpret_cast<int32_t*>(base);
+    prm.wait_limit_ns = wait_limit_ns();
+    prm.dtrace = g_dtrace;
+    return launch_gemm<ROUTE_TILED, 16>(K_ROUTE_TC, m, prm, s);
+}
+
 // ------------------------------------------------------------ linear layer
 // y [T][N] fp32 = x [T][K] . W^T for T <= 128, run as the streaming GEMM2
 // schedule with one group (weights are the M operand, the T token rows the N
@@ -1198,6 +1352,29 @@ ms_status linear_launch(const void* x, int x_rows, int T, int K, const void* w, 
 }
 
 }  // namespace ms
+
+extern "C" size_t moe_route_topk_tensor_workspace_size(int E, int H) {
+    if (E <= 0 || H <= 0) return 0;
+    return ms::route_tc_ws_bytes(E, H);
+}
+
+extern "C" ms_status moe_route_topk_tensor(const void* xhat, const float* w_router, const float* logit_bias, int T,
+                                           int H, int E, int k, int renormalize, int32_t* topk_idx, float* topk_w,
+                                           void* ws, size_t ws_bytes, void* stream) {
+    if (!xhat || !w_router || !topk_idx || !topk_w) return MS_ERR_INVALID_ARG;
+    if (T <= 0 || H <= 0 || E <= 0 || k <= 0 || k > E) return MS_ERR_INVALID_ARG;
+    if (!ms::route_tc_supported(E, k, H) || H % 128 != 0) return MS_ERR_UNSUPPORTED;
+    if (!ms::aligned16(xhat) || !ms::aligned16(w_router)) return MS_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < ms::route_tc_ws_bytes(E, H)) return MS_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 1023u) return MS_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t ce = cudaMemsetAsync(ws, 0, sizeof(int32_t), s);
+    if (ce != cudaSuccess) {
+        ms::set_cuda_error(ce);
+        return MS_ERR_CUDA;
+    }
+    return ms::route_tc_launch(xhat, w_router, logit_bias, T, H, E, k, renormalize, topk_idx, topk_w, ws, nullptr, s);
+}
 
 extern "C" size_t moe_expert_ffn_workspace_size(int T, int H, int E, int I, int S, int k) {
     if (T <= 0 || H <= 0 || E <= 0 || I <= 0 || S < 0 || k <= 0) return 0;

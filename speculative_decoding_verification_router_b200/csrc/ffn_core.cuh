@@ -36,7 +36,10 @@ constexpr int WEIGHT_BUDGET = MS_WEIGHT_BUDGET_KB * 1024;
 // this alone).
 constexpr int SMEM_CAP = 200 * 1024;
 
-enum Mode : int { G1_STREAM = 0, G2_STREAM = 1, LM_STREAM = 2, G1_TILED = 3, G2_TILED = 4 };
+enum Mode : int { G1_STREAM = 0, G2_STREAM = 1, LM_STREAM = 2, G1_TILED = 3, G2_TILED = 4, ROUTE_TILED = 5 };
+// ROUTE_TILED: the router on the tensor cores -- 128-token tiles times the
+// router weights split into three bf16 parts (N = 3E), softmax and top-k in
+// the epilogue (one thread per token).
 
 struct Maps {
     CUtensorMap w_a;     // routed weights  [E][rows][K] (or [1][V][H] for the vocab head)
@@ -61,6 +64,10 @@ struct Params {
     int nct;                       // grid size of the streaming GEMM (for the finish kernel)
     int weights_evict_first;       // streaming: weight tiles are loaded with an L2 evict-first policy
     int invariant;                 // streaming: batch-invariant schedule (whole tiles, natural k order)
+    const float* rbias;            // router (ROUTE_TILED): logit bias [T][E] or null
+    int32_t* ridx;                 //   top-k experts [T][k]
+    float* rw;                     //   their gate weights [T][k]
+    int rrenorm;                   //   divide the k weights by their sum
     int32_t* status;
     uint64_t wait_limit_ns;
     uint64_t* dtrace;              // optional per-CTA timeline (see ms_set_device_trace)
@@ -156,7 +163,7 @@ template <int MODE>
 __device__ __forceinline__ int group_ktiles(const Params& p, int g) {
     const bool shared = p.offsets != nullptr && g == p.E;
     constexpr int KS = BK * Cfg<MODE>::kSub;   // k per schedule step
-    if (MODE == G1_STREAM || MODE == G1_TILED || MODE == LM_STREAM) return p.H / KS;
+    if (MODE == G1_STREAM || MODE == G1_TILED || MODE == LM_STREAM || MODE == ROUTE_TILED) return p.H / KS;
     return (shared ? p.S * p.I : p.I) / KS;   // GEMM2: K = intermediate width
 }
 
@@ -164,6 +171,7 @@ template <int MODE>
 __device__ __forceinline__ int group_ntiles(const Params& p, int g) {
     const bool shared = p.offsets != nullptr && g == p.E;
     if (MODE == LM_STREAM) return p.V / BM;
+    if (MODE == ROUTE_TILED) return 1;
     if (MODE == G1_STREAM || MODE == G1_TILED) return (shared ? p.S * p.I : p.I) / BM;
     if (MODE == G2_STREAM) return p.H / BM;
     return p.H / p.bn;   // G2_TILED

@@ -781,14 +781,14 @@ __device__ bool lf_epilogue(const LfParams& lp, const LfRoute& rt, const Sched& 
                 }
                 continue;
             }
-            float o16[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) o16[j] = kG1 ? silu_mul(va[j], vb[j]) : va[j];
+            // static indices only: a run-time index would put the values in
+            // local memory, which (shared memory taking L1) lives in L2
             const int ncol = min(16, rows - ch * 16);
-#pragma unroll 1
-            for (int j = 0; j < ncol; ++j) {
-                if (kG1) lf_store_hv(lp, rt, sc, g, ch * 16 + j, f, o16[j]);
-                else lf_store_y(p, sc, g, ch * 16 + j, f, o16[j]);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (j >= ncol) break;
+                if (kG1) lf_store_hv(lp, rt, sc, g, ch * 16 + j, f, silu_mul(va[j], vb[j]));
+                else lf_store_y(p, sc, g, ch * 16 + j, f, va[j]);
             }
         }
         tc_fence_before();
@@ -870,12 +870,12 @@ __device__ void lf_finish1_unit(const LfParams& lp, const LfRoute& rt, const Sch
             }
     }
     const int f = n * BM + r;
-    float h[4 * NQ];
-#pragma unroll
-    for (int q = 0; q < 4 * NQ; ++q) h[q] = silu_mul(va[q], vb[q]);
     const int ncol = min(4 * NQ, sc.rows[g] - ch * 16);
-#pragma unroll 1
-    for (int q = 0; q < ncol; ++q) lf_store_hv(lp, rt, sc, g, ch * 16 + q, f, h[q]);
+#pragma unroll
+    for (int q = 0; q < 4 * NQ; ++q) {
+        if (q >= ncol) break;
+        lf_store_hv(lp, rt, sc, g, ch * 16 + q, f, silu_mul(va[q], vb[q]));
+    }
 }
 
 template <int NMAX>
@@ -1028,7 +1028,7 @@ __device__ void lf_combine(const LfParams& lp, const LfRoute& rt, const Sched& s
 // ------------------------------------------------------------ the kernel
 template <int NMAX>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    moe_layer_fused_kernel(const __grid_constant__ LfMaps mp, const LfParams lp) {
+    moe_layer_fused_kernel(const __grid_constant__ LfMaps mp, const __grid_constant__ LfParams lp) {
     using L = LfLayout<NMAX>;
     constexpr int ST = L::ST;
     const Params& p = lp.g;
@@ -1334,14 +1334,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int q_end = ring_st.qw;
         for (int s3 = 0; s3 < ST && s3 < q_end; ++s3) {
             const int q_last = s3 + ((q_end - 1 - s3) / ST) * ST;
-            volatile int never = 0;
-            if (!mbar_wait(smem_addr(&bar_full[s3]), static_cast<uint32_t>(q_last / ST) & 1u, lim, &never))
+            if (!mbar_wait(smem_addr(&bar_full[s3]), static_cast<uint32_t>(q_last / ST) & 1u, lim, nullptr))
                 drain_failed(p.status, drain_fail_sh);
         }
     } else if (threadIdx.x == 32) {
         mma_commit(smem_addr(&bar_drain));
-        volatile int never = 0;
-        if (!mbar_wait(smem_addr(&bar_drain), 0, lim, &never)) drain_failed(p.status, drain_fail_sh);
+        if (!mbar_wait(smem_addr(&bar_drain), 0, lim, nullptr)) drain_failed(p.status, drain_fail_sh);
     }
     tc_fence_before();
     __syncthreads();

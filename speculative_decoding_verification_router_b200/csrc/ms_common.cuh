@@ -37,6 +37,8 @@ enum KernelId : int {
     K_PACK,
     K_MTP_PREP,
     K_LAYER_FUSED,
+    K_ROUTE_TC,
+    K_ROUTE_SPLIT,
     K_COUNT
 };
 const char* kernel_name(int id);

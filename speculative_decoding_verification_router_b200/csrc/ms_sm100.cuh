@@ -53,7 +53,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 15u) == 0) {
-            if (*abort) return false;
+            if (abort && *abort) return false;   // null: only the time limit ends the wait
             if (global_ns() - t0 > limit_ns) return false;
         }
     }
@@ -222,7 +222,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
         if ((i & 15u) == 0) {
-            if (*abort) return false;
+            if (abort && *abort) return false;   // null: only the time limit ends the wait
             if (global_ns() - t0 > limit_ns) return false;
         }
     }

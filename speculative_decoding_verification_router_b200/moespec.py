@@ -40,6 +40,8 @@ def _load():
     sig = {
         "moe_rmsnorm": (I, [P, P, I, I, F, P, P]),
         "moe_route_topk": (I, [P, P, P, I, I, I, I, I, P, P, P]),
+        "moe_route_topk_tensor_workspace_size": (Z, [I, I]),
+        "moe_route_topk_tensor": (I, [P, P, P, I, I, I, I, I, P, P, P, Z, P]),
         "moe_permute_workspace_size": (Z, [I, I, I]),
         "moe_permute": (I, [P, I, I, I, P, P, P, P, Z, P]),
         "moe_expert_ffn_workspace_size": (Z, [I, I, I, I, I, I]),
@@ -195,6 +197,23 @@ def route_topk(xhat: torch.Tensor, w_router: torch.Tensor, bias=None, k: int = 6
                                           torch.empty((T, k), dtype=torch.float32, device=xhat.device))
     _check(_lib.moe_route_topk(_p(xhat), _p(w_router), _p(bias), T, H, E, k, int(renormalize),
                                _p(idx), _p(w), _stream(stream)), "moe_route_topk")
+    return idx, w
+
+
+def route_topk_tensor(xhat: torch.Tensor, w_router: torch.Tensor, bias=None, k: int = 6,
+                      renormalize: bool = False, ws: Optional[Workspace] = None, out=None, stream=None):
+    """The router on the tensor cores (prefill-sized batches): same results as route_topk."""
+    _dev(xhat, torch.bfloat16, "xhat")
+    _dev(w_router, torch.float32, "w_router")
+    if bias is not None:
+        _dev(bias, torch.float32, "bias")
+    T, H = xhat.shape
+    E = w_router.shape[0]
+    idx, w = out if out is not None else (torch.empty((T, k), dtype=torch.int32, device=xhat.device),
+                                          torch.empty((T, k), dtype=torch.float32, device=xhat.device))
+    wsb = _ws(ws, _lib.moe_route_topk_tensor_workspace_size(E, H), xhat.device)
+    _check(_lib.moe_route_topk_tensor(_p(xhat), _p(w_router), _p(bias), T, H, E, k, int(renormalize), _p(idx), _p(w),
+                                      wsb.c(), wsb.nbytes, _stream(stream)), "moe_route_topk_tensor")
     return idx, w
 
 

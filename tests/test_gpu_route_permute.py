@@ -52,6 +52,51 @@ def test_route_parity(ms, shp):
     np.testing.assert_allclose(host(w2).astype(np.float64).sum(1), 1.0, atol=1e-5)
 
 
+TC = [synth.MoEShape("tiny_e16", B=4, K=3, H=256, E=16, I=128, k=2, S=1, V=1024, router_std=0.05),
+      synth.VERIFY_B32, synth.PREFILL,
+      synth.MoEShape("ragged_tiles", B=1, K=0, H=1280, E=64, I=896, k=6, S=2, V=1024, router_std=0.05, tokens=1300)]
+
+
+@pytest.mark.parametrize("shp", TC, ids=[w.name for w in TC])
+def test_route_tensor_parity(ms, shp):
+    # the router on the tensor cores (three bf16 parts of W_r, fp32 accumulation):
+    # the same indices bit for bit, gates to fp32 rounding, with and without bias
+    xb, wr, bias = routed_xhat_inputs(shp, seed=0)
+    idx, w = ms.route_topk_tensor(dev(xb), dev(wr), None if bias is None else dev(bias), shp.k)
+    torch.cuda.synchronize()
+    ridx, rw, _, _ = oracle.route_topk(oracle.widen_bf16(xb), wr, bias, shp.k)
+    np.testing.assert_array_equal(host(idx), ridx)
+    np.testing.assert_allclose(host(w), rw, rtol=1e-5, atol=1e-7)
+    idx2, w2 = ms.route_topk_tensor(dev(xb), dev(wr), None if bias is None else dev(bias), shp.k, renormalize=True)
+    np.testing.assert_array_equal(host(idx2), ridx)
+    np.testing.assert_allclose(host(w2).astype(np.float64).sum(1), 1.0, atol=1e-5)
+
+
+def test_route_tensor_ties_go_to_the_lower_expert(ms):
+    # equal router rows give equal logits: the lower expert is taken first
+    T, H, E, k = 200, 256, 16, 4
+    xb = synth.normal_bf16(4, "tc_ties_x", (T, H), 1.0)
+    wr = synth.normal(4, "tc_ties_w", (E, H), 0.05)
+    wr[9] = wr[2]
+    wr[12] = wr[2]
+    wr[5] = wr[14]
+    idx, w = ms.route_topk_tensor(dev(xb), dev(wr), None, k)
+    torch.cuda.synchronize()
+    ridx, _, z, _ = oracle.route_topk(oracle.widen_bf16(xb), wr, None, k)
+    got = host(idx)
+    # where the oracle's top-k has no near-ties other than the exact duplicates, the sets agree
+    zs = -np.sort(-z.astype(np.float64), axis=1)[:, : k + 1]
+    gaps = -np.diff(zs, axis=1)
+    clear = np.all((gaps == 0) | (gaps > 1e-3), axis=1)
+    np.testing.assert_array_equal(got[clear], ridx[clear])
+    assert clear.sum() > T // 2
+    for t in np.nonzero(clear)[0]:
+        for a_, b_ in [(2, 9), (2, 12), (9, 12), (5, 14)]:
+            row = list(got[t])
+            if a_ in row and b_ in row:
+                assert row.index(a_) < row.index(b_)
+
+
 def _random_idx(T, k, E, seed, skew=None):
     g = np.random.default_rng(seed)
     p = None if skew is None else g.dirichlet(np.full(E, skew))
