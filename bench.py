@@ -254,18 +254,30 @@ def algorithmic(shp: synth.MoEShape, offsets: np.ndarray):
     return dict(active_experts=D, g1_bytes=g1_bytes, g2_bytes=g2_bytes, g1_flops=g1_flops, g2_flops=g2_flops)
 
 
-def traffic_from_profile(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source
-    still matches the one profiled (else None)."""
+def sources_sha(names):
+    """First 16 hex digits of the sha256 of the listed csrc files, concatenated in order."""
     import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "speculative_decoding_verification_router_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if every source file
+    of the kernel still matches the one profiled (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(f"{kernel}:{workload}")
     if not d:
         return None
-    src = os.path.join(ROOT, "speculative_decoding_verification_router_b200", "csrc", d["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    names = d.get("sources") or [d["source"]]
+    try:
+        h = sources_sha(names)
+    except OSError:
+        return None
     return d["bytes_per_launch"] if h == d["source_sha"] else None
 
 
@@ -406,10 +418,14 @@ def measure(shp, args, rank, world, local, device, dist, with_cpu: bool):
                      "frac": round(ach / peaks["hbm_gbs"], 4), "algorithmic_bytes": int(nb),
                      "what": "all algorithmic bytes of one step / ms_per_step", "peak_source": peaks["source"]}
     else:
+        # the step is timed in a loop of ~0.4 s, under the power cap: the sustained GEMM peak
+        # applies (the burst fraction is kept beside it)
         fl = alg["g1_flops"] + alg["g2_flops"]
         ach = fl / (ms_per_step / 1e3) / 1e12
-        roof_step = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(ach / peaks["bf16_tflops"], 4), "algorithmic_flops": int(fl),
+        sus = peaks["bf16_tflops_sustained"]
+        roof_step = {"bound": "tensor", "achieved": round(ach, 1), "peak": sus, "unit": "TFLOP/s",
+                     "frac": round(ach / sus, 4), "peak_kind": "sustained (timed in a long loop)",
+                     "frac_of_burst": round(ach / peaks["bf16_tflops"], 4), "algorithmic_flops": int(fl),
                      "what": "expert GEMM flops of one step / ms_per_step", "peak_source": peaks["source"]}
 
     # end to end through the public API with host buffers
@@ -464,6 +480,7 @@ def kernel_roofline(shp, alg, breakdown, per_kernel, peaks, wl):
     achieved = fl / dur_s / 1e12
     return {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 1),
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+            "peak_kind": "burst (kernel timed in a short traced run)",
             "traffic": traffic_from_profile(dominant, wl), "algorithmic_flops": int(fl),
             "peak_source": peaks["source"]}
 
