@@ -27,7 +27,11 @@
  *    Every call is asynchronous on that stream and never synchronises the
  *    host.  Kernels are launched with programmatic dependent launch, so a
  *    call may begin while the previous kernel on the stream drains; each
- *    kernel waits for its predecessor before touching memory.
+ *    kernel waits for its predecessor before touching activations, routing
+ *    tables, workspace or outputs.  Weights (expert, shared-expert, router
+ *    and vocabulary-head weights) are read-only inputs that kernels start
+ *    reading before that wait: they must not be written by the work that
+ *    immediately precedes the call on its stream.
  *  - Errors: arguments are validated on the host before anything is
  *    launched; a bad argument returns MS_ERR_INVALID_ARG / MS_ERR_UNSUPPORTED
  *    / MS_ERR_WORKSPACE and launches nothing.  A failed launch returns

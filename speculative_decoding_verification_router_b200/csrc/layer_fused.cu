@@ -256,21 +256,27 @@ __device__ __noinline__ void lf_load_rows(const LfParams& lp, int t0, int nt, fl
 // pairs are dealt to the warps (pair p -> expert p % ne, token p / ne), a
 // warp keeps its current router row in registers; lanes split H and a warp
 // sum finishes each dot product (a fixed order: deterministic).
-__device__ void lf_router_logits(const LfParams& lp, int e0, int ne, int t0, int nt, const float* xs) {
+// wv / cur: the warp's current router row and its expert (cur = -1: none yet;
+// the dense path loads its CTA's row before the dependency wait).
+__device__ __forceinline__ void lf_load_router_row(const LfParams& lp, int e, int lane, float4 (&wv)[LF_RWPRE]) {
+    const int H = lp.g.H;
+    const float4* wrow = reinterpret_cast<const float4*>(lp.w_router + static_cast<size_t>(e) * H);
+#pragma unroll
+    for (int j = 0; j < LF_RWPRE; ++j) {
+        const int h4 = lane + 32 * j;
+        wv[j] = h4 < H / 4 ? __ldg(wrow + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+__device__ __forceinline__ void lf_router_logits(const LfParams& lp, int e0, int ne, int t0, int nt, const float* xs,
+                                                 float4 (&wv)[LF_RWPRE], int& cur) {
     const int H = lp.g.H, E = lp.g.E;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float4 wv[LF_RWPRE];
-    int cur = -1;
 #pragma unroll 1
     for (int pidx = warp; pidx < ne * nt; pidx += LF_WARPS) {
         const int e = e0 + pidx % ne, tt = pidx / ne;
         if (e != cur) {
-            const float4* wrow = reinterpret_cast<const float4*>(lp.w_router + static_cast<size_t>(e) * H);
-#pragma unroll
-            for (int j = 0; j < LF_RWPRE; ++j) {
-                const int h4 = lane + 32 * j;
-                wv[j] = h4 < H / 4 ? __ldg(wrow + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+            lf_load_router_row(lp, e, lane, wv);
             cur = e;
         }
         const float* x = xs + tt * H;
@@ -1082,6 +1088,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         drain_fail_sh = 0;
         fence_mbar_init();
     }
+    // The router weights are read-only inputs: with at most 16 tokens CTA c's
+    // router row (expert c) is loaded now, before the dependency wait.
+    float4 wv[LF_RWPRE];
+    int wcur = -1;
+    if (lp.dense && c < E) {
+        lf_load_router_row(lp, c, lane, wv);
+        wcur = c;
+    }
     lf_prefetch_shared(lp, 0);
     // The layer input comes from the previous kernel on the stream.
     grid_dep_wait();
@@ -1100,7 +1114,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     reinterpret_cast<uint4*>(lp.x_pad + static_cast<size_t>(T) * H)[v] = make_uint4(0, 0, 0, 0);
             }
             __syncthreads();
-            for (int e = c; e < E; e += nct) lf_router_logits(lp, e, 1, 0, T, xs);
+            for (int e = c; e < E; e += nct) lf_router_logits(lp, e, 1, 0, T, xs, wv, wcur);
             if (threadIdx.x == 0) tstamp(p, 6, 1);
         }
     } else {
@@ -1135,7 +1149,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int ne = E - e0 < LF_WARPS ? E - e0 : LF_WARPS, nt = T - t0 < LF_TPI ? T - t0 : LF_TPI;
             lf_load_rows(lp, t0, nt, xs);
             __syncthreads();
-            lf_router_logits(lp, e0, ne, t0, nt, xs);
+            lf_router_logits(lp, e0, ne, t0, nt, xs, wv, wcur);
             __syncthreads();
         }
     }

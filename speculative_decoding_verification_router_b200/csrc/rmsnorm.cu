@@ -3,7 +3,11 @@
 
 namespace ms {
 
-// One warp per row; float4 loads, fp32 sum of squares, IEEE sqrt/div.
+// One warp per row; float4 loads, fp32 sum of squares, IEEE sqrt/div.  Up to
+// RN_KEEP float4 per lane (H <= 2,048) the row stays in registers between the
+// two passes, all of its loads issued at once; longer rows are read twice.
+constexpr int RN_KEEP = 16;
+
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ a,
                                                       const float* __restrict__ gamma, int T,
                                                       int H, float eps,
@@ -15,6 +19,31 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
     if (warp >= T) return;
     const float4* row = reinterpret_cast<const float4*>(a + static_cast<size_t>(warp) * H);
     const int n4 = H >> 2;
+    __nv_bfloat162* orow = reinterpret_cast<__nv_bfloat162*>(out + static_cast<size_t>(warp) * H);
+    const float4* g4 = reinterpret_cast<const float4*>(gamma);
+    if (n4 <= 32 * RN_KEEP) {
+        float4 v[RN_KEEP];
+#pragma unroll
+        for (int j = 0; j < RN_KEEP; ++j) {
+            const int i = lane + 32 * j;
+            v[j] = i < n4 ? __ldg(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < RN_KEEP; ++j) ss += v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
+        ss = warp_sum(ss);
+        const float inv = 1.0f / sqrtf(ss / static_cast<float>(H) + eps);
+#pragma unroll
+        for (int j = 0; j < RN_KEEP; ++j) {
+            const int i = lane + 32 * j;
+            if (i < n4) {
+                const float4 g = gamma ? __ldg(g4 + i) : make_float4(1.f, 1.f, 1.f, 1.f);
+                orow[2 * i] = __floats2bfloat162_rn(v[j].x * inv * g.x, v[j].y * inv * g.y);
+                orow[2 * i + 1] = __floats2bfloat162_rn(v[j].z * inv * g.z, v[j].w * inv * g.w);
+            }
+        }
+        return;
+    }
     float ss = 0.f;
     for (int i = lane; i < n4; i += 32) {
         float4 v = __ldg(row + i);
@@ -22,8 +51,6 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
     }
     ss = warp_sum(ss);
     const float inv = 1.0f / sqrtf(ss / static_cast<float>(H) + eps);
-    __nv_bfloat162* orow = reinterpret_cast<__nv_bfloat162*>(out + static_cast<size_t>(warp) * H);
-    const float4* g4 = reinterpret_cast<const float4*>(gamma);
     for (int i = lane; i < n4; i += 32) {
         float4 v = __ldg(row + i);
         float4 g = gamma ? __ldg(g4 + i) : make_float4(1.f, 1.f, 1.f, 1.f);
