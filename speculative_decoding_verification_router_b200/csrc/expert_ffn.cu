@@ -1193,10 +1193,15 @@ ms_status ffn_launch(const void* x, const int32_t* offsets, const int32_t* perm,
         if (st1 != MS_OK) return st1;
         return launch_stream<G2_STREAM>(K_GEMM2_STREAM, stream_nmax(T), m2, prm, s);
     }
-    // prefill.  GEMM2 runs as 256 x 256 tiles on CTA pairs when the output width
-    // splits in 256s (measured 638 vs 789 us at 36,992 tokens); GEMM1 stays on
-    // single CTAs, where the pair form measured slower (1,264 vs 1,212 us).
-    ms_status st = launch_gemm<G1_TILED, 16>(K_GEMM1_TILED, m1, prm, s);
+    // prefill: both GEMMs on CTA pairs, 256-token tiles.  GEMM2 (256 x 256 output
+    // tiles when the output width splits in 256s): 638 vs 789 us at 36,992
+    // tokens.  GEMM1 (256 tokens x 128 gate + 128 up features): 1,203-1,212 vs
+    // 1,246-1,279 us; each CTA stages 32 KB per k-step instead of 48 KB, which
+    // also lowers the power drawn, so the clock under the power cap is higher.
+    // MOESPEC_NO_PAIR=1 runs both on single CTAs.
+    ms_status st = (!pair_off() && pair_grid<G1_TILED>() >= 2)
+                       ? launch_gemm_pair<G1_TILED>(K_GEMM1_TILED, m1, prm, s)
+                       : launch_gemm<G1_TILED, 16>(K_GEMM1_TILED, m1, prm, s);
     if (st != MS_OK) return st;
     if (prm.bn == 256 && !pair_off() && pair_grid<G2_TILED>() >= 2)
         return launch_gemm_pair<G2_TILED>(K_GEMM2_TILED, m2, prm, s);
