@@ -944,6 +944,112 @@ __global__ void __launch_bounds__(256) ffn_prep_kernel(const __nv_bfloat16* __re
     }
 }
 
+// Prefill gather: x_perm[r] = x[perm[r]] for r < rows (the token rows in
+// expert order), rows..rows_pad-1 zero.  CTA c copies the contiguous rows
+// [c*per, (c+1)*per): their token ids are read once into shared memory, then
+// one thread streams them in chunks of R rows (R*H*2 <= 20 KB) through a ring
+// of GB_NS shared-memory slots -- a bulk load per row (the whole row) into the
+// chunk's slot and, GB_LAG chunks later, once those loads have landed, one
+// bulk store of the chunk (its rows are consecutive in x_perm).  No data
+// passes through registers, so a CTA keeps GB_LAG + 1 chunks in flight; with
+// two CTAs per SM that is about 120 KB per SM, where the warp-per-row kernel
+// keeps one row's loads per warp and waits on each row's id first.
+constexpr int GB_NS = 4, GB_LAG = 2, GB_THREADS = 128;
+static_assert(GB_LAG >= 1 && GB_LAG < GB_NS, "gather ring");
+
+__global__ void __launch_bounds__(GB_THREADS) gather_bulk_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                 const int32_t* __restrict__ perm, int T, int H,
+                                                                 int rows, int rows_pad, int per, int R,
+                                                                 __nv_bfloat16* __restrict__ x_perm,
+                                                                 int32_t* status, uint64_t lim) {
+    extern __shared__ __align__(128) uint8_t gsm[];
+    __shared__ __align__(8) uint64_t full[GB_NS];
+    const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
+    const uint32_t slot_bytes = static_cast<uint32_t>(R) * row_bytes;
+    int32_t* ids = reinterpret_cast<int32_t*>(gsm + GB_NS * slot_bytes);
+    const int r0 = static_cast<int>(blockIdx.x) * per;
+    const int r1 = min(r0 + per, rows_pad);
+    const int r1c = max(r0, min(r1, rows));   // [r0, r1c): rows with a token
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < GB_NS; ++i) mbar_init(smem_addr(&full[i]), 1);
+        fence_mbar_init();
+    }
+    grid_dep_wait();
+    grid_dep_launch();
+    // pad rows: zeros
+    const int n8 = H / 8;
+    for (long v = threadIdx.x; v < static_cast<long>(r1 - r1c) * n8; v += GB_THREADS)
+        reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(r1c) * H)[v] = make_uint4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < r1c - r0; i += GB_THREADS) {
+        int t = __ldg(perm + r0 + i);
+        if (t < 0 || t >= T) {
+            report_status(status, MS_ERR_DEVICE_INDEX);   // the row's contents are then undefined
+            t = 0;
+        }
+        ids[i] = t;
+    }
+    __syncthreads();
+    if (threadIdx.x != 0 || r1c == r0) return;
+    const int n = (r1c - r0 + R - 1) / R;
+    const uint32_t sbase = smem_addr(gsm);
+    int issued = 0, stored = 0;
+    bool ok = true;
+    for (int i = 0; i < n + GB_LAG && ok; ++i) {
+        if (i < n) {
+            // the slot's previous chunk (i - GB_NS) was stored GB_NS - 1 - GB_LAG groups ago
+            if (i >= GB_NS) bulk_wait_read<GB_NS - 1 - GB_LAG>();
+            const int sl = i % GB_NS, nr = min(R, r1c - r0 - i * R);
+            const uint32_t bar = smem_addr(&full[sl]);
+            mbar_expect_tx(bar, static_cast<uint32_t>(nr) * row_bytes);
+            for (int j = 0; j < nr; ++j)
+                bulk_load(sbase + sl * slot_bytes + j * row_bytes, x + static_cast<size_t>(ids[i * R + j]) * H,
+                          row_bytes, bar);
+            issued = i + 1;
+        }
+        const int jd = i - GB_LAG;
+        if (jd >= 0 && jd < n) {
+            const int sl = jd % GB_NS, nr = min(R, r1c - r0 - jd * R);
+            if (!mbar_wait(smem_addr(&full[sl]), static_cast<uint32_t>(jd / GB_NS) & 1u, lim, nullptr)) {
+                report_status(status, MS_ERR_TIMEOUT);
+                ok = false;
+                break;
+            }
+            bulk_store(x_perm + static_cast<size_t>(r0 + jd * R) * H, sbase + sl * slot_bytes,
+                       static_cast<uint32_t>(nr) * row_bytes);
+            bulk_commit();
+            stored = jd + 1;
+        }
+    }
+    // after a timeout: the loads still in flight land before the CTA exits (bounded)
+    for (int jd = stored; jd < issued; ++jd) {
+        if (!mbar_wait(smem_addr(&full[jd % GB_NS]), static_cast<uint32_t>(jd / GB_NS) & 1u, lim, nullptr)) {
+            report_status(status, MS_ERR_DRAIN_TIMEOUT);
+            break;
+        }
+    }
+    bulk_wait<0>();   // every store complete before the kernel ends
+}
+
+// Grid and shared memory of gather_bulk_kernel: two CTAs per SM, rows dealt in
+// contiguous ranges (a multiple of the chunk).
+struct GatherPlan {
+    int R, per, grid;
+    size_t smem;
+};
+static GatherPlan gather_plan(int H, int rows_pad) {
+    GatherPlan g{};
+    const int row_bytes = H * 2;
+    g.R = 20480 / row_bytes < 1 ? 1 : (20480 / row_bytes > 8 ? 8 : 20480 / row_bytes);
+    const int ctas = 2 * num_sms();
+    int per = (rows_pad + ctas - 1) / ctas;
+    per = (per + g.R - 1) / g.R * g.R;
+    if (per > 4096) per = 4096;   // the id table stays within 16 KB
+    g.per = per < g.R ? g.R : per;
+    g.grid = (rows_pad + g.per - 1) / g.per;
+    g.smem = static_cast<size_t>(GB_NS) * g.R * row_bytes + static_cast<size_t>(g.per) * 4;
+    return g;
+}
+
 // ------------------------------------------------------------ host side
 // MOESPEC_NO_EVICT_FIRST=1 loads the streamed weights with the default L2
 // policy (for comparison).
@@ -1077,6 +1183,15 @@ static ms_status launch_stream(int id, int nmax, const Maps& maps, const Params&
     }
 }
 
+// MOESPEC_NO_BULK_GATHER=1 gathers the prefill token rows one warp per row (for comparison).
+static bool gather_bulk_off() {
+    static const bool off = [] {
+        const char* e = getenv("MOESPEC_NO_BULK_GATHER");
+        return e && e[0] == '1';
+    }();
+    return off;
+}
+
 // MOESPEC_NO_PAIR=1 runs the prefill GEMMs on single CTAs (for comparison).
 static bool pair_off() {
     static int v = -1;
@@ -1151,8 +1266,26 @@ ms_status ffn_launch(const void* x, const int32_t* offsets, const int32_t* perm,
     FfnWs w = ffn_ws_layout(ws, T, H, E, I, S, k);
     const bool stream = T <= 128;
     const int rows = T * k;
-    // 1. gather + pad (one warp per row, 8 rows per block)
-    {
+    // 1. gather + pad: prefill through the bulk-copy ring, verify sizes one warp per row
+    if (!stream && w.rows_pad > 0 && !gather_bulk_off()) {
+        const GatherPlan g = gather_plan(H, w.rows_pad);
+        static PerDevice attr;
+        const int ok = attr.get([] {
+            const cudaError_t e =
+                cudaFuncSetAttribute(gather_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 112 * 1024);
+            if (e != cudaSuccess) {
+                set_cuda_error(e);
+                return -1;
+            }
+            return 1;
+        });
+        if (ok < 0) return MS_ERR_CUDA;
+        if (g.smem > 112 * 1024) return MS_ERR_UNSUPPORTED;
+        ms_status st = launch(K_FFN_PREP, gather_bulk_kernel, dim3(g.grid), dim3(GB_THREADS), g.smem, s,
+                              reinterpret_cast<const __nv_bfloat16*>(x), perm, T, H, rows, w.rows_pad, g.per, g.R,
+                              w.x_perm, w.status, wait_limit_ns());
+        if (st != MS_OK) return st;
+    } else {
         const long want = (static_cast<long>(w.rows_pad) + 7) / 8;
         const int grid = static_cast<int>(want < 8L * num_sms() ? want : 8L * num_sms());
         ms_status st = launch(K_FFN_PREP, ffn_prep_kernel, dim3(grid), dim3(256), 0, s,
