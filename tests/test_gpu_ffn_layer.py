@@ -120,6 +120,27 @@ def test_expert_ffn_tiled_ragged(ms, T):
     assert_close(ysh, ref["y_shared"], what="y_shared")
 
 
+def test_expert_ffn_tiled_flags_bad_token_index(ms):
+    # the prefill-sized path gathers the token rows through bulk copies:
+    # permutation entries outside [0, T) are flagged on the device and read
+    # nothing outside x; every other row is computed as usual
+    T = 300
+    shp = synth.MoEShape("tiled_badidx", B=1, K=0, H=256, E=8, I=128, k=2, S=2, V=1024, router_std=0.05, tokens=T)
+    ref, _, _ = _ffn_case(ms, shp, seed=4, y_dtype=torch.bfloat16)
+    lw = synth.layer_weights(shp, 4)
+    wgu, wd, wsgu, wsd = _weights_dev(lw)
+    bad_rows = [5, 11, T * shp.k - 1]
+    perm = ref["perm"].copy()
+    perm[bad_rows] = [T + 7, -3, 1 << 30]
+    ws = ms.Workspace(ms.expert_ffn_workspace_size(T, shp.H, shp.E, shp.I, shp.S, shp.k))
+    y, ysh = ms.expert_ffn(dev(ref["xhat_bf16"]), dev(ref["offsets"]), dev(perm), wgu, wd, wsgu, wsd, shp.k,
+                           y_dtype=torch.bfloat16, ws=ws)
+    assert ms.device_status(ws) == -6
+    keep = np.setdiff1d(np.arange(T * shp.k), bad_rows)
+    assert_close(host(y)[keep], ref["y_perm"][keep], what="y_perm rows with valid tokens")
+    assert_close(host(ysh), ref["y_shared"], what="y_shared")
+
+
 def test_expert_ffn_prefill_sampled(ms):
     # full prefill size in the launch configuration the benchmark times;
     # the oracle recomputes a sample of rows and tokens one by one
