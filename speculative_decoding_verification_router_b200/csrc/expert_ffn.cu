@@ -847,7 +847,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 template <int MODE, int NMAX>
-__global__ void __launch_bounds__(FIN_THREADS) ffn_finish_kernel(const __grid_constant__ Params p) {
+// After the gate/up GEMM at 32+ tokens the kernel is held to three CTAs' worth of
+// registers per SM: two of its CTAs and the down GEMM's CTA then share an SM.
+__global__ void __launch_bounds__(FIN_THREADS, (MODE == G1_STREAM && NMAX >= 32) ? 3 : 1) ffn_finish_kernel(const __grid_constant__ Params p) {
     __shared__ Sched sched;
     __shared__ int iprefix[MAX_GROUPS + 1];   // items before group g
     fin_stamp<MODE>(p, TS_ENTRY);

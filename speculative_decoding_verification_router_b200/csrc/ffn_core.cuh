@@ -708,9 +708,18 @@ __device__ __forceinline__ void finish_item(const Params& p, const Sched& sched,
     }
     const int rc = rows - ch * 16;   // tokens of this chunk (only those are read)
     if (kG1) {
-        if (rc <= 4) slot_sum<NMAX, 1, true>(slot_of, c_first, c_last, ch, r, va, vb);
-        else if (rc <= 8) slot_sum<NMAX, 2, true>(slot_of, c_first, c_last, ch, r, va, vb);
-        else slot_sum<NMAX, 4, true>(slot_of, c_first, c_last, ch, r, va, vb);
+        if (NMAX >= 32) {
+            // one load width (all 16 columns, whatever the chunk's tokens; the
+            // columns past them are read and never stored): one summation
+            // body keeps the kernel at ~136 registers, so the next GEMM's CTA
+            // fits beside two finish CTAs on an SM and starts its weight
+            // stream while the sums run
+            slot_sum<NMAX, 4, true>(slot_of, c_first, c_last, ch, r, va, vb);
+        } else {
+            if (rc <= 4) slot_sum<NMAX, 1, true>(slot_of, c_first, c_last, ch, r, va, vb);
+            else if (rc <= 8) slot_sum<NMAX, 2, true>(slot_of, c_first, c_last, ch, r, va, vb);
+            else slot_sum<NMAX, 4, true>(slot_of, c_first, c_last, ch, r, va, vb);
+        }
     } else {
         if (rc <= 4) slot_sum_col<1>(slot_of, c_first, c_last, ch, r, va);
         else if (rc <= 8) slot_sum_col<2>(slot_of, c_first, c_last, ch, r, va);
