@@ -1,6 +1,6 @@
 """The expert-parallel layer's partitioning, dispatch and combine on CPU.
 
-Two gloo ranks run speculative_decoding_verification_router_b200.expert_parallel
+Two or four gloo ranks run speculative_decoding_verification_router_b200.expert_parallel
 with the oracle as the per-rank compute backend (the collectives and the
 index plumbing are the module's own); the result must equal the oracle's
 single-process layer on the whole batch up to fp32 rounding of the different
@@ -127,18 +127,22 @@ def _close(got, ref):
     assert d.max() <= 1e-5 * max(np.abs(ref).max(), 1.0), d.max()
 
 
+@pytest.mark.parametrize("world", [2, 4])
 @pytest.mark.parametrize("mode", ["decode", "prefill"])
-def test_two_ranks_equal_the_whole_layer(tmp_path, mode):
+def test_ranks_equal_the_whole_layer(tmp_path, mode, world):
+    # with 4 ranks the 2 x 128 shared features go to ranks 1 and 3 only:
+    # ranks 0 and 2 hold no shared block and contribute routed rows alone
     import oracle
     oracle.build()
     port = _free_port()
-    mp.start_processes(_rank_main, args=(2, port, str(tmp_path), mode), nprocs=2, join=True, start_method="spawn")
+    mp.start_processes(_rank_main, args=(world, port, str(tmp_path), mode), nprocs=world, join=True,
+                       start_method="spawn")
     ref = _reference()
     if mode == "decode":
-        for r in range(2):
+        for r in range(world):
             _close(np.load(tmp_path / f"decode{r}.npy"), ref)
     else:
-        got = np.concatenate([np.load(tmp_path / f"prefill{r}.npy") for r in range(2)])
+        got = np.concatenate([np.load(tmp_path / f"prefill{r}.npy") for r in range(world)])
         _close(got, ref)
 
 
