@@ -277,7 +277,14 @@ MS_API ms_status spec_verify_greedy_noalloc(const void* logits, ms_dtype logits_
 /* Whole layer in hot-path order: rmsnorm -> route -> permute -> expert FFN
  * -> combine.  a: [T,H] fp32 residual input, out: [T,H] fp32.  Expert weights
  * as for moe_expert_ffn (packed).  The intermediates live in ws
- * (moe_layer_workspace_size bytes). */
+ * (moe_layer_workspace_size bytes).  Results match the five calls made one
+ * by one within the layer's tolerance (the fp32 summation order differs
+ * between the paths); how they are computed depends on T: up to 16 tokens the
+ * whole layer is one persistent kernel (unless batch-invariant schedules are
+ * set), up to 128 a chain of the weight-streaming kernels, and from 1,024
+ * tokens the router runs on the tensor cores as moe_route_topk_tensor does.
+ * Weights must not be written by the work just before the call (see the
+ * stream rule above). */
 MS_API size_t moe_layer_workspace_size(int T, int H, int E, int I, int S, int k);
 MS_API ms_status moe_layer_forward(const float* a, const float* w_router, const float* logit_bias,
                             const void* w_gate_up, const void* w_down,
