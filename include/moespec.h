@@ -153,7 +153,10 @@ MS_API ms_status moe_pack_weights(const void* w, int n, int rows, int cols, void
  * weight-streaming schedule balanced over all SMs; larger T a tiled one.
  * expert_offsets must describe groups inside [0, T*k) of at most T rows
  * each (a token reaches an expert at most once); a group that does not is
- * skipped and flagged MS_ERR_DEVICE_INDEX in the status word.
+ * skipped and flagged MS_ERR_DEVICE_INDEX in the status word, and so is a
+ * perm_token entry outside [0, T) (that row's output is then undefined).
+ * For T > 128 the token rows are staged through shared memory whole:
+ * H <= 12288 there (larger H returns MS_ERR_UNSUPPORTED).
  * Weights in the plain [E,2I,H] / [E,H,I] row-major layout (not passed
  * through moe_pack_weights) are NOT detected: both layouts hold the same
  * number of bf16 values, and the call then returns MS_OK with wrong results.
