@@ -159,6 +159,7 @@ ms_status moe_layer_forward(const float* a, const float* w_router, const float* 
     if (T <= 0 || H <= 0 || E <= 0 || I <= 0 || S < 0 || k <= 0 || k > E) return MS_ERR_INVALID_ARG;
     if (S > 0 && (!ws_gate_up || !ws_down)) return MS_ERR_INVALID_ARG;
     if (E > 256 || k > 32 || H % 128 != 0 || I % 128 != 0 || S > 8) return MS_ERR_UNSUPPORTED;
+    if (T > 128 && H > 12288) return MS_ERR_UNSUPPORTED;   // the tiled path stages whole token rows
     const ms::LayerWs w = ms::layer_layout(ws, T, H, E, I, S, k);
     if (!ws || ws_bytes < w.bytes) return MS_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(ws) & 1023u) return MS_ERR_INVALID_ARG;

@@ -72,6 +72,8 @@ def test_host_validation_rejects_bad_arguments(lib):
     lib.moe_layer_forward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, Z, P]
     assert lib.moe_layer_forward(fake, fake, None, fake, fake, fake, fake, 0, 1280, 64, 896, 2, 6, 0, fake, fake,
                                  1 << 30, None) == -1                                          # T = 0
+    assert lib.moe_layer_forward(fake, fake, None, fake, fake, fake, fake, 2048, 13312, 64, 896, 2, 6, 0, fake,
+                                 fake, 1 << 40, None) == -2                                    # prefill H > 12288
     assert lib.spec_verify_greedy(fake, 1, fake, 0, 3, 100, fake, fake, fake, fake, 1 << 20, None) == -1  # B = 0
     assert lib.spec_verify_greedy(fake, 1, None, 2, 0, 100, fake, fake, fake, None, 0, None) == -3  # K = 0 needs no drafts
     lib.moe_expert_ffn_workspace_size.restype = ctypes.c_size_t
